@@ -1,0 +1,106 @@
+"""Plant plausible mistakes in the oracle (on the CPU) and check that the pins catch each one."""
+
+import math
+
+import numpy as np
+import pytest
+
+import oracle
+import oracle.kl_oracle as ko
+import test_oracle_pins as pins
+
+
+def _fails(fn, *args):
+    try:
+        fn(*args)
+    except AssertionError:
+        return True
+    return False
+
+
+def test_swapped_mixture_weights_caught(monkeypatch):
+    monkeypatch.setattr(ko, "_log_mixture",
+                        lambda lS, lT, b: np.logaddexp(math.log(b) + lS, math.log1p(-b) + lT))
+    assert _fails(pins.test_bernoulli_v2, 0.3, -1.2)
+
+
+def test_swapped_jsd_term_weights_caught(monkeypatch):
+    orig = ko.divergence_rows
+
+    def bad(lS, lT, beta):
+        if beta in (0.0, 1.0):
+            return orig(lS, lT, beta)
+        lM = ko._log_mixture(lS, lT, beta)
+        ks, kt = ko._kl_rows(lS, lM), ko._kl_rows(lT, lM)
+        return (1 - beta) * kt + beta * ks, ks
+
+    monkeypatch.setattr(ko, "divergence_rows", bad)
+    assert _fails(pins.test_bernoulli_v2, 0.3, -1.2)
+
+
+def test_temperature_after_softmax_caught(monkeypatch):
+    orig = ko.tempered_logits
+    monkeypatch.setattr(ko, "tempered_logits", lambda h, W, tau: orig(h, W, 1.0))
+    assert _fails(pins.test_toy_v5_temperature_inside_softmax)
+
+
+def test_reversed_kl_direction_caught(monkeypatch):
+    orig = ko.divergence_rows
+    monkeypatch.setattr(ko, "divergence_rows",
+                        lambda lS, lT, b: orig(lS, lT, 1.0 - b) if b in (0.0, 1.0) else orig(lS, lT, b))
+    assert _fails(pins.test_toy_v5_tau1)
+
+
+@pytest.mark.parametrize("beta", [0.0, 1.0, 0.5])
+def test_gradient_slips_caught(monkeypatch, beta):
+    orig = ko.dloss_du_student
+
+    def dropped_term(lS, lT, b, loss, aux):
+        S = np.exp(lS)
+        if b == 0.0:
+            return np.exp(lT) - S                      # sign flipped
+        if b == 1.0:
+            return S * (lS - lT)                       # "- KL" dropped
+        return orig(lS, lT, b, loss, np.zeros_like(aux))  # "- K" dropped
+
+    monkeypatch.setattr(ko, "dloss_du_student", dropped_term)
+    assert pins._fd_check(beta, 0.7) > 1e-3
+
+
+def test_missing_inverse_tau_in_gradient_caught(monkeypatch):
+    orig = ko.backward
+
+    def bad(*a, **k):
+        out = orig(*a, **k)
+        tau = a[6]
+        out["dh_s"] *= tau
+        if out["dW_s"] is not None:
+            out["dW_s"] *= tau
+        return out
+
+    monkeypatch.setattr(oracle, "backward", bad)
+    monkeypatch.setattr(pins.oracle, "backward", bad)
+    assert pins._fd_check(1.0, 0.7) > 1e-3
+
+
+def test_mean_over_all_rows_caught(monkeypatch):
+    orig = ko.forward
+
+    def bad(*a, **k):
+        out = orig(*a, **k)
+        if out["loss_mean"] is not None and out["n_valid"]:
+            out["loss_mean"] = float(out["loss_tok"].sum() / len(a[4]))
+        return out
+
+    monkeypatch.setattr(pins.oracle, "forward", bad)
+    assert _fails(pins.test_brute_force_tiny, 1.0, 1.0)
+
+
+def test_lse_missing_log_caught(monkeypatch):
+    def bad(u):
+        m = u.max(axis=1, keepdims=True)
+        lse = m + np.exp(u - m).sum(axis=1, keepdims=True)
+        return u - lse, lse[:, 0]
+
+    monkeypatch.setattr(ko, "log_softmax", bad)
+    assert _fails(pins.test_lse_zero_weights_is_log_v)

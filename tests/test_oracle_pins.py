@@ -1,0 +1,368 @@
+"""Pins of the fp64 oracle against facts that do not come from the oracle itself.
+
+Each pin is written so that a plausible slip in the oracle (a dropped term, a wrong
+sign, a swapped beta weight, the temperature applied after the softmax, a wrong
+normaliser) makes at least one of them fail; ``test_oracle_mutations.py`` plants
+such slips and checks exactly that.
+
+Sources: "Nitrobrew tweet analysis" (sections "Nitrobrew 的两个动作", "仓库实现") and
+"03 White-box OPD" (section 1 Eq. (2), section 2.3 beta table and conventions,
+section 6 test plan).
+"""
+
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+
+import oracle
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+RTOL = 1e-12
+
+
+# ------------------------------------------------------------------ helpers
+def logits_problem(z_s, z_t, labels=None):
+    """Inputs whose logits are exactly z: h = z, W = identity (d = V)."""
+    z_s = np.atleast_2d(np.asarray(z_s, dtype=np.float64))
+    z_t = np.atleast_2d(np.asarray(z_t, dtype=np.float64))
+    V = z_s.shape[1]
+    eye = np.eye(V)
+    if labels is None:
+        labels = np.zeros(z_s.shape[0], dtype=np.int64)
+    return z_s, eye, z_t, eye.copy(), np.asarray(labels, dtype=np.int64)
+
+
+def fwd(z_s, z_t, beta, tau=1.0, labels=None):
+    return oracle.forward(*logits_problem(z_s, z_t, labels), beta, tau)
+
+
+def rand_problem(rng, N, V, d_s, d_t, scale=1.0):
+    h_s = rng.standard_normal((N, d_s))
+    h_t = rng.standard_normal((N, d_t))
+    W_s = rng.standard_normal((V, d_s)) * scale / math.sqrt(d_s)
+    W_t = rng.standard_normal((V, d_t)) * scale / math.sqrt(d_t)
+    return h_s, W_s, h_t, W_t
+
+
+# ------------------------------------------------------------------ pure-Python brute force
+def brute_row(hs, Ws, ht, Wt, beta, tau):
+    """Probability-domain evaluation with explicit loops (no max shift, no log-sum-exp)."""
+    V = len(Ws)
+    zs = [math.fsum(a * b for a, b in zip(hs, Ws[v])) / tau for v in range(V)]
+    zt = [math.fsum(a * b for a, b in zip(ht, Wt[v])) / tau for v in range(V)]
+    es, et = [math.exp(x) for x in zs], [math.exp(x) for x in zt]
+    Zs, Zt = math.fsum(es), math.fsum(et)
+    S, T = [e / Zs for e in es], [e / Zt for e in et]
+    if beta == 0.0:
+        loss = math.fsum(T[v] * math.log(T[v] / S[v]) for v in range(V))
+    elif beta == 1.0:
+        loss = math.fsum(S[v] * math.log(S[v] / T[v]) for v in range(V))
+    else:
+        M = [(1 - beta) * S[v] + beta * T[v] for v in range(V)]
+        loss = beta * math.fsum(T[v] * math.log(T[v] / M[v]) for v in range(V)) + \
+            (1 - beta) * math.fsum(S[v] * math.log(S[v] / M[v]) for v in range(V))
+    return loss, math.log(Zs), math.log(Zt)
+
+
+@pytest.mark.parametrize("beta", [0.0, 1.0, 0.5, 0.2, 0.9])
+@pytest.mark.parametrize("tau", [1.0, 0.7, 2.0])
+def test_brute_force_tiny(beta, tau):
+    rng = np.random.default_rng(11)
+    N, V, d_s, d_t = 4, 13, 5, 7
+    h_s, W_s, h_t, W_t = rand_problem(rng, N, V, d_s, d_t, scale=2.0)
+    labels = np.array([3, -100, 0, 12])
+    out = oracle.forward(h_s, W_s, h_t, W_t, labels, beta, tau)
+    acc = []
+    for n in range(N):
+        if labels[n] == -100:
+            assert out["loss_tok"][n] == 0.0
+            continue
+        loss, ls, lt = brute_row(h_s[n], W_s, h_t[n], W_t, beta, tau)
+        assert out["loss_tok"][n] == pytest.approx(loss, rel=1e-11, abs=1e-14)
+        assert out["lse_s"][n] == pytest.approx(ls, rel=RTOL)
+        assert out["lse_t"][n] == pytest.approx(lt, rel=RTOL)
+        acc.append(loss)
+    assert out["n_valid"] == 3
+    assert out["loss_mean"] == pytest.approx(math.fsum(acc) / 3, rel=1e-11)
+
+
+def test_lse_brute_force_v64():
+    rng = np.random.default_rng(3)
+    h_s, W_s, h_t, W_t = rand_problem(rng, 5, 64, 8, 8, scale=4.0)
+    out = oracle.forward(h_s, W_s, h_t, W_t, np.zeros(5, np.int64), 1.0, 1.3)
+    for n in range(5):
+        _, ls, lt = brute_row(h_s[n], W_s, h_t[n], W_t, 1.0, 1.3)
+        assert out["lse_s"][n] == pytest.approx(ls, rel=RTOL)
+        assert out["lse_t"][n] == pytest.approx(lt, rel=RTOL)
+
+
+def test_lse_zero_weights_is_log_v():
+    V = 37
+    out = oracle.forward(np.ones((2, 3)), np.zeros((V, 3)), np.ones((2, 4)), np.zeros((V, 4)),
+                         np.zeros(2, np.int64), 1.0, 1.0)
+    np.testing.assert_allclose(out["lse_s"], math.log(V), rtol=RTOL)
+    np.testing.assert_allclose(out["loss_tok"], 0.0, atol=1e-15)
+
+
+# ------------------------------------------------------------------ closed forms
+def test_uniform_teacher_closed_forms():
+    rng = np.random.default_rng(5)
+    V = 50
+    z_s = rng.standard_normal((3, V)) * 3
+    z_t = np.zeros((3, V))
+    rev = fwd(z_s, z_t, 1.0)["loss_tok"]
+    fkl = fwd(z_s, z_t, 0.0)["loss_tok"]
+    for n in range(3):
+        e = [math.exp(x) for x in z_s[n]]
+        Z = math.fsum(e)
+        S = [x / Z for x in e]
+        H = -math.fsum(p * math.log(p) for p in S)
+        assert rev[n] == pytest.approx(math.log(V) - H, rel=1e-12)
+        assert fkl[n] == pytest.approx(-math.log(V) - math.fsum(math.log(p) for p in S) / V, rel=1e-12)
+
+
+@pytest.mark.parametrize("a,b", [(0.3, -1.2), (4.0, 2.5), (-3.0, 3.0)])
+def test_bernoulli_v2(a, b):
+    s = 1 / (1 + math.exp(-a))
+    t = 1 / (1 + math.exp(-b))
+    z_s, z_t = [[a, 0.0]], [[b, 0.0]]
+    rev = s * math.log(s / t) + (1 - s) * math.log((1 - s) / (1 - t))
+    fkl = t * math.log(t / s) + (1 - t) * math.log((1 - t) / (1 - s))
+    assert fwd(z_s, z_t, 1.0)["loss_tok"][0] == pytest.approx(rev, rel=1e-12)
+    assert fwd(z_s, z_t, 0.0)["loss_tok"][0] == pytest.approx(fkl, rel=1e-12)
+    beta = 0.3
+    m = (1 - beta) * s + beta * t
+    jsd = beta * (t * math.log(t / m) + (1 - t) * math.log((1 - t) / (1 - m))) + \
+        (1 - beta) * (s * math.log(s / m) + (1 - s) * math.log((1 - s) / (1 - m)))
+    assert fwd(z_s, z_t, beta)["loss_tok"][0] == pytest.approx(jsd, rel=1e-12)
+
+
+def _toy():
+    with open(os.path.join(GOLDEN, "toy_v5.json")) as f:
+        g = json.load(f)
+    return g["student_weights"], g["teacher_weights"]
+
+
+def test_toy_v5_tau1():
+    ws, wt = _toy()
+    S = [x / sum(ws) for x in ws]
+    T = [x / sum(wt) for x in wt]
+    assert S == [0.05, 0.1, 0.15, 0.2, 0.5] and T == [0.1, 0.1, 0.1, 0.1, 0.6]
+    z_s, z_t = [np.log(ws)], [np.log(wt)]
+    # hand-expanded: sum_v S_v ln(S_v / T_v) etc., with the ratios written out
+    rev = 0.05 * math.log(0.5) + 0.15 * math.log(1.5) + 0.2 * math.log(2.0) + 0.5 * math.log(5 / 6)
+    fkl = 0.1 * math.log(2.0) + 0.1 * math.log(2 / 3) + 0.1 * math.log(0.5) + 0.6 * math.log(1.2)
+    M = [0.075, 0.1, 0.125, 0.15, 0.55]
+    jsd = 0.5 * (0.1 * math.log(0.1 / 0.075) + 0.1 * math.log(0.1 / 0.125) + 0.1 * math.log(0.1 / 0.15)
+                 + 0.6 * math.log(0.6 / 0.55)) + \
+        0.5 * (0.05 * math.log(0.05 / 0.075) + 0.15 * math.log(0.15 / 0.125) + 0.2 * math.log(0.2 / 0.15)
+               + 0.5 * math.log(0.5 / 0.55))
+    assert fwd(z_s, z_t, 1.0)["loss_tok"][0] == pytest.approx(rev, rel=1e-13)
+    assert fwd(z_s, z_t, 0.0)["loss_tok"][0] == pytest.approx(fkl, rel=1e-13)
+    assert fwd(z_s, z_t, 0.5)["loss_tok"][0] == pytest.approx(jsd, rel=1e-13)
+    assert fwd(z_s, z_t, 1.0)["lse_s"][0] == pytest.approx(math.log(20.0), rel=1e-14)
+
+
+def test_toy_v5_temperature_inside_softmax():
+    """softmax(z / tau) is sqrt(weights) normalised at tau = 2, not softmax(z) / tau."""
+    ws, wt = _toy()
+    rs, rt = [math.sqrt(x) for x in ws], [math.sqrt(x) for x in wt]
+    S = [x / math.fsum(rs) for x in rs]
+    T = [x / math.fsum(rt) for x in rt]
+    rev = math.fsum(S[v] * math.log(S[v] / T[v]) for v in range(5))
+    got = fwd([np.log(ws)], [np.log(wt)], 1.0, tau=2.0)
+    assert got["loss_tok"][0] == pytest.approx(rev, rel=1e-12)
+    assert got["lse_s"][0] == pytest.approx(math.log(math.fsum(rs)), rel=1e-13)
+    # the wrong placement (divide the probabilities by tau) gives a different number
+    S1 = [x / sum(ws) for x in ws]
+    T1 = [x / sum(wt) for x in wt]
+    wrong = math.fsum((S1[v] / 2) * math.log(S1[v] / T1[v]) for v in range(5))
+    assert abs(got["loss_tok"][0] - wrong) > 1e-3
+
+
+# ------------------------------------------------------------------ invariants
+@pytest.mark.parametrize("beta", [0.0, 1.0, 0.5, 0.25])
+def test_nonnegative_and_zero_when_equal(beta):
+    rng = np.random.default_rng(7)
+    h_s, W_s, h_t, W_t = rand_problem(rng, 16, 40, 6, 9, scale=3.0)
+    labels = np.zeros(16, np.int64)
+    out = oracle.forward(h_s, W_s, h_t, W_t, labels, beta, 1.0)
+    assert (out["loss_tok"] > 0).all()
+    same = oracle.forward(h_s, W_s, h_s, W_s, labels, beta, 1.0)
+    np.testing.assert_allclose(same["loss_tok"], 0.0, atol=1e-14)
+    back = oracle.backward(h_s, W_s, h_s, W_s, labels, beta, 1.0)
+    np.testing.assert_allclose(back["dh_s"], 0.0, atol=1e-15)
+    np.testing.assert_allclose(back["dW_s"], 0.0, atol=1e-15)
+
+
+def test_swap_symmetries():
+    rng = np.random.default_rng(8)
+    h_s, W_s, h_t, W_t = rand_problem(rng, 10, 30, 6, 6, scale=3.0)
+    lab = np.zeros(10, np.int64)
+    f = oracle.forward(h_s, W_s, h_t, W_t, lab, 0.0, 1.1)["loss_tok"]
+    r = oracle.forward(h_t, W_t, h_s, W_s, lab, 1.0, 1.1)["loss_tok"]
+    np.testing.assert_allclose(f, r, rtol=1e-12)
+    j = oracle.forward(h_s, W_s, h_t, W_t, lab, 0.3, 1.1)["loss_tok"]
+    js = oracle.forward(h_t, W_t, h_s, W_s, lab, 0.7, 1.1)["loss_tok"]
+    np.testing.assert_allclose(j, js, rtol=1e-12)
+    # the directions differ in general
+    assert np.abs(f - oracle.forward(h_s, W_s, h_t, W_t, lab, 1.0, 1.1)["loss_tok"]).max() > 1e-3
+
+
+@pytest.mark.parametrize("beta", [0.5, 0.1, 0.8])
+def test_jsd_bound_and_disjoint_limit(beta):
+    hb = -beta * math.log(beta) - (1 - beta) * math.log(1 - beta)
+    assert hb <= math.log(2) + 1e-15
+    rng = np.random.default_rng(9)
+    V = 40
+    z_s = rng.standard_normal((6, V)) * 4
+    z_t = rng.standard_normal((6, V)) * 4
+    out = fwd(z_s, z_t, beta)["loss_tok"]
+    assert (out >= 0).all() and (out <= hb).all()
+    # one-hot peaks at different ids: JSD -> h(beta)
+    z_s = np.zeros((1, V)); z_s[0, 3] = 60.0
+    z_t = np.zeros((1, V)); z_t[0, 17] = 60.0
+    assert fwd(z_s, z_t, beta)["loss_tok"][0] == pytest.approx(hb, rel=1e-9)
+
+
+def test_jsd_half_matches_scipy():
+    from scipy.spatial.distance import jensenshannon
+    rng = np.random.default_rng(10)
+    V = 33
+    z_s = rng.standard_normal((4, V)) * 2
+    z_t = rng.standard_normal((4, V)) * 2
+    got = fwd(z_s, z_t, 0.5)["loss_tok"]
+    for n in range(4):
+        p = np.exp(z_s[n]) / np.exp(z_s[n]).sum()
+        q = np.exp(z_t[n]) / np.exp(z_t[n]).sum()
+        assert got[n] == pytest.approx(jensenshannon(p, q) ** 2, rel=1e-10)
+
+
+def test_temperature_scaling_invariance_and_limit():
+    rng = np.random.default_rng(12)
+    h_s, W_s, h_t, W_t = rand_problem(rng, 5, 20, 4, 4, scale=3.0)
+    lab = np.zeros(5, np.int64)
+    for beta in (0.0, 1.0, 0.5):
+        a = oracle.forward(h_s, W_s, h_t, W_t, lab, beta, 1.5)["loss_tok"]
+        b = oracle.forward(3.0 * h_s, W_s, 3.0 * h_t, W_t, lab, beta, 4.5)["loss_tok"]
+        np.testing.assert_allclose(a, b, rtol=1e-12)
+        big = oracle.forward(h_s, W_s, h_t, W_t, lab, beta, 1e6)["loss_tok"]
+        assert big.max() < 1e-9
+
+
+def test_direction_confident_vs_diffuse():
+    """Reverse KL punishes student mass where a confident teacher has none; forward KL the converse."""
+    V = 5
+    eps = 1e-6
+    peaked = np.log([1 - eps] + [eps / (V - 1)] * (V - 1))
+    flat = np.zeros(V)
+    # diffuse student, confident teacher
+    r1 = fwd([flat], [peaked], 1.0)["loss_tok"][0]
+    f1 = fwd([flat], [peaked], 0.0)["loss_tok"][0]
+    assert r1 > f1
+    # confident student, diffuse teacher
+    r2 = fwd([peaked], [flat], 1.0)["loss_tok"][0]
+    f2 = fwd([peaked], [flat], 0.0)["loss_tok"][0]
+    assert f2 > r2
+
+
+# ------------------------------------------------------------------ reduction and masking
+def test_per_token_mean_masking_permutation():
+    rng = np.random.default_rng(13)
+    N = 9
+    h_s, W_s, h_t, W_t = rand_problem(rng, N, 21, 5, 6, scale=2.5)
+    labels = np.array([1, -100, 4, 4, -100, -100, 0, 2, 7])
+    out = oracle.forward(h_s, W_s, h_t, W_t, labels, 1.0, 1.0)
+    valid = labels != -100
+    assert out["n_valid"] == 6
+    assert out["loss_mean"] == pytest.approx(out["loss_tok"][valid].sum() / 6, rel=1e-14)
+    assert (out["loss_tok"][~valid] == 0).all() and (out["lse_s"][~valid] == 0).all()
+    # the mean is not the sum and not the mean over all N rows
+    assert out["loss_mean"] != pytest.approx(out["loss_tok"].sum() / N, rel=1e-6)
+    back = oracle.backward(h_s, W_s, h_t, W_t, labels, 1.0, 1.0)
+    assert (back["dh_s"][~valid] == 0).all()
+    perm = rng.permutation(N)
+    outp = oracle.forward(h_s[perm], W_s, h_t[perm], W_t, labels[perm], 1.0, 1.0)
+    np.testing.assert_allclose(outp["loss_tok"], out["loss_tok"][perm], rtol=1e-14)
+    backp = oracle.backward(h_s[perm], W_s, h_t[perm], W_t, labels[perm], 1.0, 1.0)
+    np.testing.assert_allclose(backp["dh_s"], back["dh_s"][perm], rtol=1e-12, atol=1e-18)
+    np.testing.assert_allclose(backp["dW_s"], back["dW_s"], rtol=1e-10, atol=1e-16)
+
+
+def test_no_valid_rows():
+    rng = np.random.default_rng(14)
+    h_s, W_s, h_t, W_t = rand_problem(rng, 4, 10, 3, 3)
+    labels = np.full(4, -100)
+    out = oracle.forward(h_s, W_s, h_t, W_t, labels, 1.0, 1.0)
+    assert out["n_valid"] == 0 and out["loss_mean"] == 0.0
+    back = oracle.backward(h_s, W_s, h_t, W_t, labels, 1.0, 1.0)
+    assert not back["dh_s"].any() and not back["dW_s"].any()
+
+
+# ------------------------------------------------------------------ gradients
+def _fd_check(beta, tau, seed=0):
+    rng = np.random.default_rng(100 + seed)
+    N, V, d = 3, 7, 4
+    h_s, W_s, h_t, W_t = rand_problem(rng, N, V, d, d + 1, scale=2.0)
+    labels = np.array([2, -100, 5])
+    grad_out = 0.7
+
+    def L(hs, ws):
+        return grad_out * oracle.forward(hs, ws, h_t, W_t, labels, beta, tau)["loss_mean"]
+
+    back = oracle.backward(h_s, W_s, h_t, W_t, labels, beta, tau, grad_out=grad_out)
+    eps = 1e-6
+    worst = 0.0
+    for arr, g, which in ((h_s, back["dh_s"], 0), (W_s, back["dW_s"], 1)):
+        num = np.zeros_like(arr)
+        for idx in np.ndindex(*arr.shape):
+            p, m = arr.copy(), arr.copy()
+            p[idx] += eps
+            m[idx] -= eps
+            lp = L(p, W_s) if which == 0 else L(h_s, p)
+            lm = L(m, W_s) if which == 0 else L(h_s, m)
+            num[idx] = (lp - lm) / (2 * eps)
+        worst = max(worst, np.abs(num - g).max() / np.abs(num).max())
+    return worst
+
+
+@pytest.mark.parametrize("beta", [0.0, 1.0, 0.5, 0.3])
+@pytest.mark.parametrize("tau", [0.7, 2.0])
+def test_finite_difference_gradients(beta, tau):
+    assert _fd_check(beta, tau) < 1e-6
+
+
+def test_gradient_row_sums_vanish():
+    """Softmax shift invariance: sum_v G[n, v] = 0, hence the column sums of dW_s vanish."""
+    rng = np.random.default_rng(15)
+    h_s, W_s, h_t, W_t = rand_problem(rng, 6, 25, 5, 7, scale=3.0)
+    lab = np.zeros(6, np.int64)
+    for beta in (0.0, 1.0, 0.4):
+        back = oracle.backward(h_s, W_s, h_t, W_t, lab, beta, 1.2)
+        colsum = back["dW_s"].sum(axis=0)
+        assert np.abs(colsum).max() < 1e-14 * max(1.0, np.abs(back["dW_s"]).max() * 25)
+        # <dW_s, W_s> = <dh_s, h_s> (both equal sum G * z_s)
+        assert np.sum(back["dW_s"] * W_s) == pytest.approx(np.sum(back["dh_s"] * h_s), rel=1e-10)
+
+
+def test_reverse_kl_gradient_blows_up_as_teacher_prob_vanishes():
+    """03 White-box OPD, section 1 (gradient blow-up) and section 6 item 1."""
+    V = 8
+    z_s = np.zeros((1, V))
+    z_s[0, 2] = 1.0
+    base = np.linspace(-1, 1, V)
+    R = np.exp(np.delete(base, 2)).sum()
+    norms = []
+    for p in [1e-1, 1e-2, 1e-3, 1e-4, 1e-5, 1e-6]:
+        z_t = base.copy()
+        z_t[2] = math.log(p * R / (1 - p))
+        out = fwd(z_s, [z_t], 1.0)
+        T2 = math.exp(z_t[2] - out["lse_t"][0])
+        assert T2 == pytest.approx(p, rel=1e-9)
+        g = oracle.backward(*logits_problem(z_s, [z_t]), 1.0, 1.0)["dh_s"]
+        norms.append(np.linalg.norm(g))
+    assert all(b > a for a, b in zip(norms, norms[1:]))
+    assert norms[-1] > 3 * norms[0]
