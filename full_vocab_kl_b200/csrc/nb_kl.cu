@@ -1,0 +1,507 @@
+// C-ABI host layer: argument checks, workspace carve-up, TMA descriptors, launches.
+//
+// One forward call: compaction of the valid rows -> vocabulary sweep (both block GEMMs,
+// online LSE / KL epilogue, split-V partial state) -> split-V merge -> [JSD: second
+// sweep with the final LSEs -> partial-sum reduction] -> masked mean.
+// One backward call: compaction -> per vocabulary chunk { gradient sweep writing the bf16
+// gradient chunk G; grouped GEMM dh_s (+)= G W_s[chunk], dW_s[chunk] (+)= G^T h_s }.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/nb_kl.h"
+#include "common.cuh"
+#include "gemm.cuh"
+#include "rowops.cuh"
+#include "sweep.cuh"
+
+using namespace nbkl;
+
+namespace {
+
+constexpr unsigned long long kWaitLimitNs = 1000000000ull;  // 1 s per pipeline wait
+constexpr int kTilesPerUnitFwd = 16;                         // 2048 vocabulary columns per split
+constexpr int64_t kDefaultChunkV = 8192;
+constexpr size_t kCtrlBytes = 256;
+
+thread_local int g_launches = 0;
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+int64_t round_up(int64_t x, int64_t m) { return (x + m - 1) / m * m; }
+
+struct Layout {
+  int64_t N, N_pad, V, d_s, d_t;
+  int split;             // fp32 hidden states stored as [hi | lo] bf16
+  int kb_s, kb_t;        // 64-wide K blocks of W
+  int64_t lda_s, lda_t;  // row length of the compacted h buffers
+  int n_vt, n_split;
+  int64_t chunk_v;
+  size_t off_idx, off_hs, off_ht, off_rl2s, off_rl2t, off_raux, off_state, off_part, off_G, total;
+  long long fs_state;    // elements between state fields
+};
+
+bool make_layout(const nb_kl_shape* sh, float beta, Layout& L) {
+  if (!sh) return false;
+  if (sh->n_tokens < 0 || sh->vocab < 1 || sh->d_s < 8 || sh->d_t < 8) return false;
+  if (sh->d_s % 8 || sh->d_t % 8) return false;
+  if (sh->h_dtype != NB_BF16 && sh->h_dtype != NB_F32) return false;
+  if (sh->reserved != 0) return false;
+  if (sh->chunk_v < 0 || (sh->chunk_v % 128) != 0) return false;
+  if (sh->n_tokens > (int64_t(1) << 30) || sh->vocab > (int64_t(1) << 30) || sh->d_s > 65536 || sh->d_t > 65536)
+    return false;
+  L.N = sh->n_tokens;
+  L.N_pad = round_up(std::max<int64_t>(L.N, 1), kBlockM);
+  L.V = sh->vocab;
+  L.d_s = sh->d_s;
+  L.d_t = sh->d_t;
+  L.split = sh->h_dtype == NB_F32;
+  L.kb_s = int((L.d_s + kBlockK - 1) / kBlockK);
+  L.kb_t = int((L.d_t + kBlockK - 1) / kBlockK);
+  L.lda_s = int64_t(L.kb_s) * kBlockK * (L.split ? 2 : 1);
+  L.lda_t = int64_t(L.kb_t) * kBlockK * (L.split ? 2 : 1);
+  L.n_vt = int((L.V + kBlockN - 1) / kBlockN);
+  L.n_split = (L.n_vt + kTilesPerUnitFwd - 1) / kTilesPerUnitFwd;
+  L.chunk_v = sh->chunk_v ? sh->chunk_v : std::min<int64_t>(kDefaultChunkV, round_up(L.V, kBlockN));
+  const bool jsd = beta > 0.f && beta < 1.f;
+  size_t off = kCtrlBytes;
+  L.off_idx = off;   off = align256(off + size_t(L.N_pad) * 4);
+  L.off_hs = off;    off = align256(off + size_t(L.N_pad) * L.lda_s * 2);
+  L.off_ht = off;    off = align256(off + size_t(L.N_pad) * L.lda_t * 2);
+  L.off_rl2s = off;  off = align256(off + size_t(L.N_pad) * 4);
+  L.off_rl2t = off;  off = align256(off + size_t(L.N_pad) * 4);
+  L.off_raux = off;  off = align256(off + size_t(L.N_pad) * 4);
+  // the forward's split state and the backward's gradient chunk share one region
+  const size_t state_bytes = align256(size_t(5) * L.n_split * L.N_pad * 4);
+  const size_t part_bytes = jsd ? align256(size_t(2) * L.n_split * L.N_pad * 4) : 0;
+  const size_t g_bytes = align256(size_t(L.N_pad) * L.chunk_v * 2);
+  L.off_state = off;
+  L.off_part = off + state_bytes;
+  L.off_G = off;
+  off += std::max(state_bytes + part_bytes, g_bytes);
+  L.total = off;
+  L.fs_state = (long long)L.n_split * L.N_pad;
+  return true;
+}
+
+// ------------------------------------------------------------------ device / driver set-up
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  std::call_once(g_encode_once, [] {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &fn, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  });
+  return g_encode;
+}
+
+struct DevInfo {
+  int sms = 0;
+  bool ok = false;
+  bool attrs = false;
+};
+DevInfo g_dev[64];
+std::mutex g_dev_mu;
+
+nb_status device_info(DevInfo& out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return NB_ERR_CUDA;
+  std::lock_guard<std::mutex> lk(g_dev_mu);
+  DevInfo& d = g_dev[dev];
+  if (!d.attrs) {
+    int major = 0, sms = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) return NB_ERR_CUDA;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return NB_ERR_CUDA;
+    d.sms = sms;
+    d.ok = major == 10;
+    if (d.ok) {
+      bool fail = false;
+      fail |= cudaFuncSetAttribute(sweep_kernel<kStateNone>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes) != cudaSuccess;
+      fail |= cudaFuncSetAttribute(sweep_kernel<kStateS>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes) != cudaSuccess;
+      fail |= cudaFuncSetAttribute(sweep_kernel<kStateT>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes) != cudaSuccess;
+      fail |= cudaFuncSetAttribute(sweep_kernel<kJsd>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes) != cudaSuccess;
+      fail |= cudaFuncSetAttribute(sweep_kernel<kGradFkl>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes) != cudaSuccess;
+      fail |= cudaFuncSetAttribute(sweep_kernel<kGradRkl>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes) != cudaSuccess;
+      fail |= cudaFuncSetAttribute(sweep_kernel<kGradJsd>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes) != cudaSuccess;
+      fail |= cudaFuncSetAttribute(gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes) != cudaSuccess;
+      if (fail) return NB_ERR_CUDA;
+    }
+    d.attrs = true;
+  }
+  out = d;
+  return d.ok ? NB_OK : NB_ERR_UNSUPPORTED;
+}
+
+// 2-D bf16 tensor map with 128-byte swizzle; out-of-range elements read as zero.
+bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint64_t row_bytes,
+              uint32_t box_inner, uint32_t box_outer) {
+  auto enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {row_bytes};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t es[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+template <typename K, typename... Args>
+void launch(K kernel, dim3 grid, dim3 block, size_t smem, cudaStream_t st, Args... args) {
+  kernel<<<grid, block, smem, st>>>(args...);
+  ++g_launches;
+}
+
+nb_status check_launch() { return cudaGetLastError() == cudaSuccess ? NB_OK : NB_ERR_CUDA; }
+
+struct Ws {
+  Ctrl* ctrl;
+  int* idx;
+  __nv_bfloat16 *hs, *ht;
+  float *rl2s, *rl2t, *raux, *state, *part;
+  __nv_bfloat16* G;
+};
+
+Ws carve(const Layout& L, void* ws) {
+  uint8_t* b = static_cast<uint8_t*>(ws);
+  Ws w;
+  w.ctrl = reinterpret_cast<Ctrl*>(b);
+  w.idx = reinterpret_cast<int*>(b + L.off_idx);
+  w.hs = reinterpret_cast<__nv_bfloat16*>(b + L.off_hs);
+  w.ht = reinterpret_cast<__nv_bfloat16*>(b + L.off_ht);
+  w.rl2s = reinterpret_cast<float*>(b + L.off_rl2s);
+  w.rl2t = reinterpret_cast<float*>(b + L.off_rl2t);
+  w.raux = reinterpret_cast<float*>(b + L.off_raux);
+  w.state = reinterpret_cast<float*>(b + L.off_state);
+  w.part = reinterpret_cast<float*>(b + L.off_part);
+  w.G = reinterpret_cast<__nv_bfloat16*>(b + L.off_G);
+  return w;
+}
+
+void launch_gather(const Layout& L, const Ws& w, const void* h, int64_t d, __nv_bfloat16* dst, int64_t lda,
+                   cudaStream_t st, const float* lse_s = nullptr, const float* lse_t = nullptr,
+                   const float* aux = nullptr) {
+  const int half = int(lda / (L.split ? 2 : 1));
+  float *r2s = nullptr, *r2t = nullptr, *rax = nullptr;
+  if (lse_s) {
+    r2s = w.rl2s;
+    r2t = w.rl2t;
+    rax = w.raux;
+  }
+  if (L.split)
+    launch(gather_rows_kernel<true>, dim3(unsigned(L.N_pad)), dim3(128), 0, st, h, int(d), dst, int(lda), half,
+           (const int*)w.idx, (const Ctrl*)w.ctrl, lse_s, lse_t, aux, r2s, r2t, rax);
+  else
+    launch(gather_rows_kernel<false>, dim3(unsigned(L.N_pad)), dim3(128), 0, st, h, int(d), dst, int(lda), half,
+           (const int*)w.idx, (const Ctrl*)w.ctrl, lse_s, lse_t, aux, r2s, r2t, rax);
+}
+
+bool sweep_maps(const Layout& L, const Ws& w, const void* W_s, const void* W_t, SweepMaps& m) {
+  bool ok = true;
+  ok &= make_map(&m.a_s, w.hs, L.lda_s, L.N_pad, L.lda_s * 2, kBlockK, kBlockM);
+  ok &= make_map(&m.b_s, W_s, L.d_s, L.V, L.d_s * 2, kBlockK, kBlockN);
+  ok &= make_map(&m.a_t, w.ht, L.lda_t, L.N_pad, L.lda_t * 2, kBlockK, kBlockM);
+  ok &= make_map(&m.b_t, W_t, L.d_t, L.V, L.d_t * 2, kBlockK, kBlockN);
+  return ok;
+}
+
+SweepArgs base_sweep_args(const Layout& L, const Ws& w, float beta, float tau) {
+  SweepArgs a;
+  std::memset(&a, 0, sizeof(a));
+  a.V = int(L.V);
+  a.v_begin = 0;
+  a.v_end = int(L.V);
+  a.nkb_s = int(L.lda_s / kBlockK);
+  a.nkb_t = int(L.lda_t / kBlockK);
+  a.bmod_s = L.kb_s;
+  a.bmod_t = L.kb_t;
+  a.tiles_per_unit = kTilesPerUnitFwd;
+  a.scale = float(1.4426950408889634 / double(tau));
+  a.beta = beta;
+  a.lg2_1mb = (beta < 1.f) ? float(std::log2(1.0 - double(beta))) : 0.f;
+  a.lg2_b = (beta > 0.f) ? float(std::log2(double(beta))) : 0.f;
+  a.ld = int(L.N_pad);
+  a.field_stride = L.fs_state;
+  a.row_l2s = w.rl2s;
+  a.row_l2t = w.rl2t;
+  a.row_aux = w.raux;
+  a.n_valid = &w.ctrl->n_valid;
+  a.gscale = &w.ctrl->gscale;
+  a.status = &w.ctrl->status;
+  a.wait_limit_ns = kWaitLimitNs;
+  return a;
+}
+
+int sweep_grid(const DevInfo& dev, const Layout& L, const SweepArgs& a) {
+  const int n_tt = int(L.N_pad / kBlockM);
+  const int n_vt = (a.v_end - a.v_begin + kBlockN - 1) / kBlockN;
+  const int n_vu = (n_vt + a.tiles_per_unit - 1) / a.tiles_per_unit;
+  return std::max(1, std::min(dev.sms, n_tt * n_vu));
+}
+
+template <int MODE>
+void launch_sweep(const DevInfo& dev, const Layout& L, const SweepMaps& m, const SweepArgs& a, cudaStream_t st) {
+  launch(sweep_kernel<MODE>, dim3(sweep_grid(dev, L, a)), dim3(kThreads), size_t(kSmemBytes), st, m, a);
+}
+
+nb_status validate_common(const nb_kl_shape* shape, const void* h_s, const void* W_s, const void* h_t,
+                          const void* W_t, const int64_t* labels, float beta, float tau, void* workspace,
+                          size_t ws_bytes, Layout& L) {
+  if (!make_layout(shape, beta, L)) return NB_ERR_INVALID_ARG;
+  if (!(beta >= 0.f && beta <= 1.f)) return NB_ERR_INVALID_ARG;
+  if (!(tau > 0.f) || !std::isfinite(tau)) return NB_ERR_INVALID_ARG;
+  if (!workspace || !aligned16(workspace)) return NB_ERR_INVALID_ARG;
+  if (L.N > 0) {
+    if (!h_s || !W_s || !h_t || !W_t || !labels) return NB_ERR_INVALID_ARG;
+    if (!aligned16(h_s) || !aligned16(W_s) || !aligned16(h_t) || !aligned16(W_t)) return NB_ERR_INVALID_ARG;
+  }
+  if (ws_bytes < L.total) return NB_ERR_WORKSPACE;
+  return NB_OK;
+}
+
+}  // namespace
+
+// =====================================================================================
+extern "C" {
+
+size_t nb_kl_workspace_size(const nb_kl_shape* shape, float beta) {
+  Layout L;
+  if (!make_layout(shape, beta, L)) return 0;
+  return L.total;
+}
+
+const char* nb_kl_status_string(nb_status s) {
+  switch (s) {
+    case NB_OK: return "ok";
+    case NB_ERR_INVALID_ARG: return "invalid argument";
+    case NB_ERR_UNSUPPORTED: return "unsupported device or size";
+    case NB_ERR_WORKSPACE: return "workspace too small";
+    case NB_ERR_CUDA: return "CUDA error";
+    case NB_ERR_TIMEOUT: return "device wait timed out";
+  }
+  return "unknown status";
+}
+
+int nb_kl_last_launch_count(void) { return g_launches; }
+
+nb_status nb_kl_device_status(void* workspace, void* stream) {
+  if (!workspace) return NB_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int status = 0;
+  if (cudaMemcpyAsync(&status, workspace, sizeof(int), cudaMemcpyDeviceToHost, st) != cudaSuccess)
+    return NB_ERR_CUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return NB_ERR_CUDA;
+  return static_cast<nb_status>(status);
+}
+
+nb_status nb_kl_forward(const nb_kl_shape* shape, const void* h_s, const void* W_s, const void* h_t,
+                        const void* W_t, const int64_t* labels, float beta, float tau, float* loss_tok,
+                        float* lse_s, float* lse_t, float* aux, float* loss_mean, int64_t* n_valid,
+                        void* workspace, size_t workspace_bytes, void* stream) {
+  g_launches = 0;
+  Layout L;
+  nb_status s = validate_common(shape, h_s, W_s, h_t, W_t, labels, beta, tau, workspace, workspace_bytes, L);
+  if (s != NB_OK) return s;
+  if (!loss_mean || !n_valid) return NB_ERR_INVALID_ARG;
+  if (L.N > 0 && (!loss_tok || !lse_s || !lse_t || !aux)) return NB_ERR_INVALID_ARG;
+  DevInfo dev;
+  if ((s = device_info(dev)) != NB_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const Ws w = carve(L, workspace);
+  if (cudaMemsetAsync(w.ctrl, 0, kCtrlBytes, st) != cudaSuccess) return NB_ERR_CUDA;
+  if (L.N == 0) {
+    if (cudaMemsetAsync(loss_mean, 0, sizeof(float), st) != cudaSuccess) return NB_ERR_CUDA;
+    if (cudaMemsetAsync(n_valid, 0, sizeof(int64_t), st) != cudaSuccess) return NB_ERR_CUDA;
+    return NB_OK;
+  }
+  const size_t nb = size_t(L.N) * sizeof(float);
+  if (cudaMemsetAsync(loss_tok, 0, nb, st) != cudaSuccess || cudaMemsetAsync(lse_s, 0, nb, st) != cudaSuccess ||
+      cudaMemsetAsync(lse_t, 0, nb, st) != cudaSuccess || cudaMemsetAsync(aux, 0, nb, st) != cudaSuccess)
+    return NB_ERR_CUDA;
+
+  launch(compact_kernel, dim3(1), dim3(kScanThreads), 0, st, labels, int(L.N), (long long)shape->ignore_index,
+         w.idx, w.ctrl, n_valid, (const float*)nullptr, tau);
+  launch_gather(L, w, h_s, L.d_s, w.hs, L.lda_s, st);
+  launch_gather(L, w, h_t, L.d_t, w.ht, L.lda_t, st);
+
+  SweepMaps maps;
+  if (!sweep_maps(L, w, W_s, W_t, maps)) return NB_ERR_CUDA;
+  SweepArgs a = base_sweep_args(L, w, beta, tau);
+  a.out = w.state;
+  int kl_dir = 0;
+  if (beta == 1.f) {
+    launch_sweep<kStateS>(dev, L, maps, a, st);
+    kl_dir = 1;
+  } else if (beta == 0.f) {
+    launch_sweep<kStateT>(dev, L, maps, a, st);
+    kl_dir = 2;
+  } else {
+    launch_sweep<kStateNone>(dev, L, maps, a, st);
+  }
+  const unsigned rb = unsigned((L.N_pad + 255) / 256);
+  launch(merge_kernel, dim3(rb), dim3(256), 0, st, (const float*)w.state, (long long)L.fs_state, int(L.N_pad),
+         L.n_split, (const int*)w.idx, (const Ctrl*)w.ctrl, kl_dir, loss_tok, lse_s, lse_t, aux, w.rl2s, w.rl2t);
+  if (kl_dir == 0) {
+    SweepArgs b = a;
+    b.out = w.part;
+    launch_sweep<kJsd>(dev, L, maps, b, st);
+    launch(jsd_finalize_kernel, dim3(rb), dim3(256), 0, st, (const float*)w.part, (long long)L.fs_state,
+           int(L.N_pad), L.n_split, (const int*)w.idx, (const Ctrl*)w.ctrl, loss_tok, aux);
+  }
+  launch(mean_kernel, dim3(1), dim3(1024), 0, st, (const float*)loss_tok, int(L.N), (const Ctrl*)w.ctrl,
+         loss_mean);
+  return check_launch();
+}
+
+nb_status nb_kl_backward(const nb_kl_shape* shape, const void* h_s, const void* W_s, const void* h_t,
+                         const void* W_t, const int64_t* labels, float beta, float tau, const float* lse_s,
+                         const float* lse_t, const float* aux, const float* grad_out, float* dh_s, float* dW_s,
+                         int accumulate_dW, void* workspace, size_t workspace_bytes, void* stream) {
+  g_launches = 0;
+  Layout L;
+  nb_status s = validate_common(shape, h_s, W_s, h_t, W_t, labels, beta, tau, workspace, workspace_bytes, L);
+  if (s != NB_OK) return s;
+  if (!dW_s || !grad_out) return NB_ERR_INVALID_ARG;
+  if (!aligned16(dW_s)) return NB_ERR_INVALID_ARG;
+  if (L.N > 0 && (!lse_s || !lse_t || !aux || !dh_s || !aligned16(dh_s))) return NB_ERR_INVALID_ARG;
+  DevInfo dev;
+  if ((s = device_info(dev)) != NB_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const Ws w = carve(L, workspace);
+  if (cudaMemsetAsync(w.ctrl, 0, kCtrlBytes, st) != cudaSuccess) return NB_ERR_CUDA;
+  if (L.N == 0) {
+    if (!accumulate_dW && cudaMemsetAsync(dW_s, 0, size_t(L.V) * L.d_s * 4, st) != cudaSuccess) return NB_ERR_CUDA;
+    return NB_OK;
+  }
+  launch(compact_kernel, dim3(1), dim3(kScanThreads), 0, st, labels, int(L.N), (long long)shape->ignore_index,
+         w.idx, w.ctrl, (int64_t*)nullptr, grad_out, tau);
+  launch_gather(L, w, h_s, L.d_s, w.hs, L.lda_s, st, lse_s, lse_t, aux);
+  launch_gather(L, w, h_t, L.d_t, w.ht, L.lda_t, st);
+  launch(zero_masked_rows_kernel, dim3(unsigned(L.N)), dim3(128), 0, st, labels, (long long)shape->ignore_index,
+         dh_s, int(L.d_s));
+
+  SweepMaps maps;
+  if (!sweep_maps(L, w, W_s, W_t, maps)) return NB_ERR_CUDA;
+  GemmMaps gm;
+  bool ok = true;
+  // dh_s: A = G (K-major, box 64 x 128), B = W_s chunk as K x N (MN-major, 64 x 64 boxes)
+  ok &= make_map(&gm.a[0], w.G, L.chunk_v, L.N_pad, L.chunk_v * 2, kBlockK, kBlockM);
+  ok &= make_map(&gm.b[0], W_s, L.d_s, L.V, L.d_s * 2, 64, 64);
+  // dW_s: A = G^T (MN-major), B = compacted h_s (hi part) as K x N (MN-major)
+  ok &= make_map(&gm.a[1], w.G, L.chunk_v, L.N_pad, L.chunk_v * 2, 64, 64);
+  ok &= make_map(&gm.b[1], w.hs, L.d_s, L.N_pad, L.lda_s * 2, 64, 64);
+  if (!ok) return NB_ERR_CUDA;
+
+  SweepArgs a = base_sweep_args(L, w, beta, tau);
+  a.G = w.G;
+  a.ldG = L.chunk_v;
+  a.tiles_per_unit = 1;
+  GemmArgs g;
+  std::memset(&g, 0, sizeof(g));
+  g.nprob = 2;
+  g.n_valid = &w.ctrl->n_valid;
+  g.status = &w.ctrl->status;
+  g.wait_limit_ns = kWaitLimitNs;
+  GemmProb& dh = g.prob[0];
+  dh.a_mn = 0;
+  dh.b_mn = 1;
+  dh.m_dyn = 1;
+  dh.N = int(L.d_s);
+  dh.out = dh_s;
+  dh.ldo = L.d_s;
+  dh.row_map = w.idx;
+  GemmProb& dw = g.prob[1];
+  dw.a_mn = 1;
+  dw.b_mn = 1;
+  dw.N = int(L.d_s);
+  dw.k_dyn = 1;
+  dw.ldo = L.d_s;
+  dw.accumulate = accumulate_dW ? 1 : 0;
+
+  const int n_tt_max = int(L.N_pad / kBlockM);
+  const int n_dt = int((L.d_s + kBlockN - 1) / kBlockN);
+  for (int64_t v0 = 0; v0 < L.V; v0 += L.chunk_v) {
+    const int64_t v1 = std::min(L.V, v0 + L.chunk_v);
+    a.v_begin = int(v0);
+    a.v_end = int(v1);
+    if (beta == 0.f) launch_sweep<kGradFkl>(dev, L, maps, a, st);
+    else if (beta == 1.f) launch_sweep<kGradRkl>(dev, L, maps, a, st);
+    else launch_sweep<kGradJsd>(dev, L, maps, a, st);
+    dh.K = int(v1 - v0);
+    dh.b_koff = int(v0);
+    dh.accumulate = v0 > 0 ? 1 : 0;
+    dw.M = int(v1 - v0);
+    dw.out = dW_s + v0 * L.d_s;
+    const int tiles = n_tt_max * n_dt + int((v1 - v0 + kBlockM - 1) / kBlockM) * n_dt;
+    launch(gemm_kernel, dim3(std::max(1, std::min(dev.sms, tiles))), dim3(kThreads), size_t(kSmemBytes), st, gm, g);
+  }
+  return check_launch();
+}
+
+nb_status nb_kl_debug_gemm(const void* A, int a_mn_major, const void* B, int b_mn_major, int64_t M, int64_t N,
+                           int64_t K, float* C, void* workspace, void* stream) {
+  g_launches = 0;
+  if (!A || !B || !C || !workspace) return NB_ERR_INVALID_ARG;
+  if (M < 1 || N < 1 || K < 1 || M % 8 || N % 8 || K % 8) return NB_ERR_INVALID_ARG;
+  if (M > (1 << 30) || N > (1 << 30) || K > (1 << 30)) return NB_ERR_INVALID_ARG;
+  if (!aligned16(A) || !aligned16(B) || !aligned16(C) || !aligned16(workspace)) return NB_ERR_INVALID_ARG;
+  DevInfo dev;
+  nb_status s = device_info(dev);
+  if (s != NB_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  Ctrl* ctrl = static_cast<Ctrl*>(workspace);
+  if (cudaMemsetAsync(ctrl, 0, kCtrlBytes, st) != cudaSuccess) return NB_ERR_CUDA;
+  GemmMaps gm;
+  std::memset(&gm, 0, sizeof(gm));
+  bool ok = true;
+  if (!a_mn_major) ok &= make_map(&gm.a[0], A, K, M, K * 2, kBlockK, kBlockM);
+  else ok &= make_map(&gm.a[0], A, M, K, M * 2, 64, 64);
+  if (!b_mn_major) ok &= make_map(&gm.b[0], B, K, N, K * 2, kBlockK, kBlockN);
+  else ok &= make_map(&gm.b[0], B, N, K, N * 2, 64, 64);
+  if (!ok) return NB_ERR_CUDA;
+  GemmArgs g;
+  std::memset(&g, 0, sizeof(g));
+  g.nprob = 1;
+  g.n_valid = &ctrl->n_valid;
+  g.status = &ctrl->status;
+  g.wait_limit_ns = kWaitLimitNs;
+  GemmProb& q = g.prob[0];
+  q.a_mn = a_mn_major ? 1 : 0;
+  q.b_mn = b_mn_major ? 1 : 0;
+  q.M = int(M);
+  q.N = int(N);
+  q.K = int(K);
+  q.out = C;
+  q.ldo = N;
+  const int tiles = int((M + kBlockM - 1) / kBlockM * ((N + kBlockN - 1) / kBlockN));
+  launch(gemm_kernel, dim3(std::max(1, std::min(dev.sms, tiles))), dim3(kThreads), size_t(kSmemBytes), st, gm, g);
+  return check_launch();
+}
+
+nb_status nb_kl_debug_wait_timeout(void* workspace, uint64_t limit_ns, void* stream) {
+  g_launches = 0;
+  if (!workspace || !aligned16(workspace)) return NB_ERR_INVALID_ARG;
+  if (limit_ns > 5000000000ull) return NB_ERR_INVALID_ARG;
+  DevInfo dev;
+  nb_status s = device_info(dev);
+  if (s != NB_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(workspace, 0, kCtrlBytes, st) != cudaSuccess) return NB_ERR_CUDA;
+  launch(wait_timeout_kernel, dim3(1), dim3(32), 0, st, &static_cast<Ctrl*>(workspace)->status,
+         (unsigned long long)limit_ns);
+  return check_launch();
+}
+
+}  // extern "C"

@@ -1,0 +1,388 @@
+// Vocabulary sweep: both block GEMMs on tcgen05 with a fused per-token epilogue.
+//
+// "Nitrobrew tweet analysis", section "Nitrobrew 的两个动作": for each vocabulary
+// block, z_s = h_s W_s[v0:v1]^T and z_t = h_t W_t[v0:v1]^T are formed, the online
+// softmax / log-sum-exp accumulators and the KL terms are updated, and the block is
+// discarded. Here one block is a 128-token x 128-column tile: the student and the
+// teacher accumulators (128 TMEM columns each) live side by side in tensor memory,
+// double-buffered so that the epilogue of tile j overlaps the MMAs of tile j + 1.
+//
+// Warp roles (192 threads, one CTA per SM, persistent over work units):
+//   warp 0  TMA producer: h and W tiles into a 6-stage shared-memory ring
+//   warp 1  MMA issuer: 4 x tcgen05.mma (K = 16) per 64-wide K block; owns TMEM
+//   warps 2-5  epilogue: tcgen05.ld of one token row per thread, base-2 online math
+//
+// A work unit is (token tile, run of `tiles_per_unit` vocabulary tiles); its per-token
+// partial state is written once per unit (the split-V partial LSE state).
+#pragma once
+
+#include "common.cuh"
+
+namespace nbkl {
+
+struct SweepSmem {
+  uint8_t* a;          // kStages x 16 KB
+  uint8_t* b;          // kStages x 16 KB
+  uint64_t* full;      // kStages
+  uint64_t* empty;     // kStages
+  uint64_t* tfull;     // 2
+  uint64_t* tempty;    // 2
+  uint64_t* drain;     // 1
+  uint32_t* tmem_slot;
+};
+
+__device__ __forceinline__ SweepSmem carve_smem(uint8_t* raw) {
+  SweepSmem s;
+  uint8_t* base = align1024(raw);
+  s.a = base;
+  s.b = base + kStages * kTileBytes;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(base + kStages * kStageBytes);
+  s.full = bars;
+  s.empty = bars + kStages;
+  s.tfull = bars + 2 * kStages;
+  s.tempty = bars + 2 * kStages + 2;
+  s.drain = bars + 2 * kStages + 4;
+  s.tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * kStages + 5);
+  return s;
+}
+
+struct UnitGrid {
+  int n_valid, n_tt, n_vt, n_vu, n_units;
+};
+
+__device__ __forceinline__ UnitGrid unit_grid(const SweepArgs& p) {
+  UnitGrid g;
+  g.n_valid = *p.n_valid;
+  g.n_tt = (g.n_valid + kBlockM - 1) / kBlockM;
+  g.n_vt = (p.v_end - p.v_begin + kBlockN - 1) / kBlockN;
+  g.n_vu = (g.n_vt + p.tiles_per_unit - 1) / p.tiles_per_unit;
+  g.n_units = g.n_tt * g.n_vu;
+  return g;
+}
+
+// ------------------------------------------------------------------ producer
+__device__ __forceinline__ void sweep_producer(const SweepMaps& maps, const SweepArgs& p, const UnitGrid& g,
+                                               const SweepSmem& s, const WaitCtl& w) {
+  int stage = 0;
+  uint32_t phase = 0;
+  const int nkb = p.nkb_s + p.nkb_t;
+  uint32_t pend_stage[kStages];
+  uint32_t pend_par[kStages];
+  int n_issued = 0;
+  bool ok = true;
+  for (int u = blockIdx.x; u < g.n_units && ok; u += gridDim.x) {
+    const int vu = u / g.n_tt, tt = u % g.n_tt;
+    const int t_end = min((vu + 1) * p.tiles_per_unit, g.n_vt);
+    for (int t = vu * p.tiles_per_unit; t < t_end && ok; ++t) {
+      const int v0 = p.v_begin + t * kBlockN;
+      for (int kb = 0; kb < nkb; ++kb) {
+        if (!mbar_wait(&s.empty[stage], phase ^ 1u, w)) { ok = false; break; }
+        const bool stu = kb < p.nkb_s;
+        const int k = stu ? kb : kb - p.nkb_s;
+        const int kbb = k % (stu ? p.bmod_s : p.bmod_t);
+        const uint32_t bar = smem_addr(&s.full[stage]);
+        mbar_arrive_expect_tx(&s.full[stage], kStageBytes);
+        tma_load_2d(smem_addr(s.a + stage * kTileBytes), stu ? &maps.a_s : &maps.a_t, bar, k * kBlockK,
+                    tt * kBlockM);
+        tma_load_2d(smem_addr(s.b + stage * kTileBytes), stu ? &maps.b_s : &maps.b_t, bar, kbb * kBlockK, v0);
+        pend_stage[n_issued % kStages] = stage;
+        pend_par[n_issued % kStages] = phase;
+        ++n_issued;
+        if (++stage == kStages) { stage = 0; phase ^= 1u; }
+      }
+    }
+  }
+  if (!ok) {
+    // drain: wait (bounded) for the copies still in flight before the CTA can exit
+    const int n = min(n_issued, kStages);
+    for (int i = 0; i < n; ++i) {
+      const int j = (n_issued - 1 - i) % kStages;
+      const uint32_t a = smem_addr(&s.full[pend_stage[j]]);
+      const uint64_t t0 = global_timer_ns();
+      while (!mbar_test(a, pend_par[j]) && global_timer_ns() - t0 < 100000000ull) {
+      }
+    }
+  }
+}
+
+// ------------------------------------------------------------------ MMA issuer
+__device__ __forceinline__ void sweep_mma(const SweepArgs& p, const UnitGrid& g, const SweepSmem& s,
+                                          uint32_t tmem_base, const WaitCtl& w) {
+  int stage = 0;
+  uint32_t phase = 0;
+  int acc = 0;
+  uint32_t acc_phase = 0;
+  const int nkb = p.nkb_s + p.nkb_t;
+  bool ok = true;
+  for (int u = blockIdx.x; u < g.n_units && ok; u += gridDim.x) {
+    const int vu = u / g.n_tt;
+    const int t_end = min((vu + 1) * p.tiles_per_unit, g.n_vt);
+    for (int t = vu * p.tiles_per_unit; t < t_end && ok; ++t) {
+      if (!mbar_wait(&s.tempty[acc], acc_phase ^ 1u, w)) { ok = false; break; }
+      tc_fence_after();
+      const uint32_t d_s = tmem_base + acc * 256;
+      for (int kb = 0; kb < nkb; ++kb) {
+        if (!mbar_wait(&s.full[stage], phase, w)) { ok = false; break; }
+        tc_fence_after();
+        const bool stu = kb < p.nkb_s;
+        const int k = stu ? kb : kb - p.nkb_s;
+        const uint32_t d = stu ? d_s : d_s + 128;
+        const uint32_t sa = smem_addr(s.a + stage * kTileBytes);
+        const uint32_t sb = smem_addr(s.b + stage * kTileBytes);
+#pragma unroll
+        for (int j = 0; j < kBlockK / 16; ++j) {
+          umma_bf16(d, make_sdesc(sa + j * 32, 16, 1024), make_sdesc(sb + j * 32, 16, 1024), kIdescKK,
+                    (k > 0 || j > 0) ? 1u : 0u);
+        }
+        umma_commit(smem_addr(&s.empty[stage]));
+        if (++stage == kStages) { stage = 0; phase ^= 1u; }
+      }
+      if (!ok) break;
+      umma_commit(smem_addr(&s.tfull[acc]));
+      acc ^= 1;
+      if (acc == 0) acc_phase ^= 1u;
+    }
+  }
+  if (!ok) {
+    // make sure no MMA still writes TMEM before it is released
+    umma_commit(smem_addr(s.drain));
+    const uint32_t a = smem_addr(s.drain);
+    const uint64_t t0 = global_timer_ns();
+    while (!mbar_test(a, 0) && global_timer_ns() - t0 < 100000000ull) {
+    }
+  }
+}
+
+// ------------------------------------------------------------------ epilogue math
+// Online base-2 state of one token row: running maxima m, rescaled sums l = sum 2^(x - m),
+// and a = sum 2^(x_p - m_p) (x_p - x_q) for the model p the KL takes its expectation under.
+struct RowState {
+  float ms, ls, mt, lt, a;
+};
+
+template <int MODE, bool MASKED>
+__device__ __forceinline__ void chunk_state(float (&zs)[32], float (&zt)[32], int n_ok, float scale, RowState& r) {
+  float cs = kNegBig, ct = kNegBig;
+#pragma unroll
+  for (int j = 0; j < 32; ++j) {
+    float xs = zs[j] * scale, xt = zt[j] * scale;
+    if (MASKED && j >= n_ok) { xs = kNegBig; xt = kNegBig; }
+    zs[j] = xs;
+    zt[j] = xt;
+    cs = fmaxf(cs, xs);
+    ct = fmaxf(ct, xt);
+  }
+  const float ns = fmaxf(r.ms, cs), nt = fmaxf(r.mt, ct);
+  const float rs = ex2(r.ms - ns), rt = ex2(r.mt - nt);
+  r.ls *= rs;
+  r.lt *= rt;
+  if (MODE == kStateS) r.a *= rs;
+  if (MODE == kStateT) r.a *= rt;
+  r.ms = ns;
+  r.mt = nt;
+  float ls = 0.f, lt = 0.f, a = 0.f;
+#pragma unroll
+  for (int j = 0; j < 32; ++j) {
+    const float es = ex2(zs[j] - ns);
+    const float et = ex2(zt[j] - nt);
+    ls += es;
+    lt += et;
+    if (MODE == kStateS) a = fmaf(es, zs[j] - zt[j], a);
+    if (MODE == kStateT) a = fmaf(et, zt[j] - zs[j], a);
+  }
+  r.ls += ls;
+  r.lt += lt;
+  r.a += a;
+}
+
+struct RowConst {
+  float l2s, l2t, aux;
+  float beta, omb, lg2_1mb, lg2_b;
+};
+
+// log2 of the mixture M = (1 - beta) S + beta T from base-2 log-probabilities.
+__device__ __forceinline__ float log2_mixture(float ys, float yt, const RowConst& c) {
+  const float a = ys + c.lg2_1mb, b = yt + c.lg2_b;
+  const float hi = fmaxf(a, b), lo = fminf(a, b);
+  return hi + lg2(1.0f + ex2(lo - hi));
+}
+
+template <bool MASKED>
+__device__ __forceinline__ void chunk_jsd(const float (&zs)[32], const float (&zt)[32], int n_ok, float scale,
+                                          const RowConst& c, float& js, float& ks) {
+  float j_acc = 0.f, k_acc = 0.f;
+#pragma unroll
+  for (int j = 0; j < 32; ++j) {
+    const float ys = fmaf(zs[j], scale, -c.l2s);
+    const float yt = fmaf(zt[j], scale, -c.l2t);
+    float S = ex2(ys), T = ex2(yt);
+    if (MASKED && j >= n_ok) { S = 0.f; T = 0.f; }
+    const float ym = log2_mixture(ys, yt, c);
+    const float ds = ys - ym, dt = yt - ym;
+    k_acc = fmaf(S, ds, k_acc);
+    j_acc = fmaf(c.beta * T, dt, j_acc);
+  }
+  // JSD = beta * KL(T||M) + (1 - beta) * KL(S||M); the S term is the K accumulator
+  js += j_acc + c.omb * k_acc;
+  ks += k_acc;
+}
+
+// d loss_n / d u_s for one element, base-2 inputs.
+template <int MODE>
+__device__ __forceinline__ float grad_elem(float xs, float xt, const RowConst& c) {
+  const float ys = xs - c.l2s, yt = xt - c.l2t;
+  const float S = ex2(ys);
+  if (MODE == kGradFkl) return S - ex2(yt);
+  if (MODE == kGradRkl) return S * fmaf(kLn2, ys - yt, -c.aux);
+  const float ym = log2_mixture(ys, yt, c);
+  return c.omb * S * fmaf(kLn2, ys - ym, -c.aux);
+}
+
+template <int MODE, bool MASKED>
+__device__ __forceinline__ void chunk_grad(const float (&zs)[32], const float (&zt)[32], int n_ok, float scale,
+                                           const RowConst& c, float gs, __nv_bfloat16* dst) {
+  uint32_t packed[16];
+#pragma unroll
+  for (int j = 0; j < 32; j += 2) {
+    float g0 = gs * grad_elem<MODE>(zs[j] * scale, zt[j] * scale, c);
+    float g1 = gs * grad_elem<MODE>(zs[j + 1] * scale, zt[j + 1] * scale, c);
+    if (MASKED && j >= n_ok) g0 = 0.f;
+    if (MASKED && j + 1 >= n_ok) g1 = 0.f;
+    __nv_bfloat162 h = __floats2bfloat162_rn(g0, g1);
+    packed[j / 2] = *reinterpret_cast<uint32_t*>(&h);
+  }
+  uint4* d4 = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+  for (int q = 0; q < 4; ++q)
+    d4[q] = make_uint4(packed[4 * q], packed[4 * q + 1], packed[4 * q + 2], packed[4 * q + 3]);
+}
+
+// ------------------------------------------------------------------ epilogue
+template <int MODE>
+__device__ __forceinline__ void sweep_epilogue(const SweepArgs& p, const UnitGrid& g, const SweepSmem& s,
+                                               uint32_t tmem_base, const WaitCtl& w) {
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int q = warp & 3;                      // TMEM lane quarter this warp may access
+  const int row_in_tile = q * 32 + lane;
+  const uint32_t lane_addr = uint32_t(q * 32) << 16;
+  int acc = 0;
+  uint32_t acc_phase = 0;
+  RowConst c;
+  c.beta = p.beta;
+  c.omb = 1.0f - p.beta;
+  c.lg2_1mb = p.lg2_1mb;
+  c.lg2_b = p.lg2_b;
+  const float gscale = (MODE >= kGradFkl) ? *p.gscale : 0.f;
+
+  for (int u = blockIdx.x; u < g.n_units; u += gridDim.x) {
+    const int vu = u / g.n_tt, tt = u % g.n_tt;
+    const int row = tt * kBlockM + row_in_tile;
+    const bool row_ok = row < g.n_valid;
+    if (MODE >= kJsd) {
+      c.l2s = p.row_l2s[row];
+      c.l2t = p.row_l2t[row];
+      c.aux = p.row_aux[row];
+    }
+    const float gs = row_ok ? gscale : 0.f;
+    RowState r{kNegBig, 0.f, kNegBig, 0.f, 0.f};
+    float js = 0.f, ks = 0.f;
+    const int t_end = min((vu + 1) * p.tiles_per_unit, g.n_vt);
+    for (int t = vu * p.tiles_per_unit; t < t_end; ++t) {
+      const int v0 = p.v_begin + t * kBlockN;
+      if (!mbar_wait(&s.tfull[acc], acc_phase, w)) return;
+      tc_fence_after();
+      const uint32_t base = tmem_base + lane_addr + acc * 256;
+#pragma unroll 1
+      for (int ch = 0; ch < 4; ++ch) {
+        float zs[32], zt[32];
+        tmem_ld32(base + ch * 32, zs);
+        tmem_ld32(base + 128 + ch * 32, zt);
+        tmem_wait_ld();
+        if (ch == 3) {
+          tc_fence_before();
+          mbar_arrive(&s.tempty[acc]);
+        }
+        const int c0 = v0 + ch * 32;
+        const int n_ok = p.V - c0;          // columns of this chunk inside the vocabulary
+        const bool masked = n_ok < 32;
+        if (MODE <= kStateT) {
+          if (masked) chunk_state<MODE, true>(zs, zt, n_ok, p.scale, r);
+          else chunk_state<MODE, false>(zs, zt, n_ok, p.scale, r);
+        } else if (MODE == kJsd) {
+          if (masked) chunk_jsd<true>(zs, zt, n_ok, p.scale, c, js, ks);
+          else chunk_jsd<false>(zs, zt, n_ok, p.scale, c, js, ks);
+        } else {
+          __nv_bfloat16* dst = p.G + (long long)row * p.ldG + (c0 - p.v_begin);
+          if (masked) chunk_grad<MODE, true>(zs, zt, n_ok, p.scale, c, gs, dst);
+          else chunk_grad<MODE, false>(zs, zt, n_ok, p.scale, c, gs, dst);
+        }
+      }
+      acc ^= 1;
+      if (acc == 0) acc_phase ^= 1u;
+    }
+    const long long off = (long long)vu * p.ld + row;
+    if (MODE <= kStateT) {
+      p.out[off] = r.ms;
+      p.out[p.field_stride + off] = r.ls;
+      p.out[2 * p.field_stride + off] = r.mt;
+      p.out[3 * p.field_stride + off] = r.lt;
+      p.out[4 * p.field_stride + off] = r.a;
+    } else if (MODE == kJsd) {
+      p.out[off] = js;
+      p.out[p.field_stride + off] = ks;
+    }
+  }
+}
+
+template <int MODE>
+__global__ void __launch_bounds__(kThreads, 1)
+    sweep_kernel(const __grid_constant__ SweepMaps maps, const SweepArgs p) {
+  extern __shared__ uint8_t smem_raw[];
+  const SweepSmem s = carve_smem(smem_raw);
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kStages; ++i) {
+      mbar_init(&s.full[i], 1);
+      mbar_init(&s.empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&s.tfull[i], 1);
+      mbar_init(&s.tempty[i], kEpiThreads);
+    }
+    mbar_init(s.drain, 1);
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_map(&maps.a_s);
+    tma_prefetch_map(&maps.b_s);
+    tma_prefetch_map(&maps.a_t);
+    tma_prefetch_map(&maps.b_t);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_addr(s.tmem_slot), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *s.tmem_slot;
+  const UnitGrid g = unit_grid(p);
+  const WaitCtl w{p.status, p.wait_limit_ns};
+
+  if (warp == 0) {
+    if (lane == 0) sweep_producer(maps, p, g, s, w);
+  } else if (warp == 1) {
+    if (lane == 0) sweep_mma(p, g, s, tmem_base, w);
+  } else {
+    sweep_epilogue<MODE>(p, g, s, tmem_base, w);
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem_base, 512);
+  }
+}
+
+}  // namespace nbkl

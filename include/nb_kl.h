@@ -1,0 +1,127 @@
+/*
+ * nb_kl — full-vocabulary hidden-state distillation loss on NVIDIA B200 (sm_100a).
+ *
+ * C ABI. Every pointer argument named h_*, W_*, labels, loss_*, lse_*, aux, n_valid,
+ * grad_out, dh_s, dW_s and workspace is a DEVICE pointer; shapes are passed by value in
+ * a host-side nb_kl_shape. Nothing here allocates device memory: the caller owns every
+ * buffer, including the workspace. All calls are asynchronous on `stream` (a
+ * cudaStream_t passed as void*; NULL = legacy default stream).
+ *
+ * What is computed ("Nitrobrew tweet analysis", sections "Nitrobrew 的两个动作" and
+ * "工程落地"; "03 White-box OPD", sections 1 and 2.3):
+ *   z_s = h_s W_s^T, z_t = h_t W_t^T, rebuilt one vocabulary block at a time and never
+ *   stored; u = z / tau (temperature inside the softmax); S = softmax(u_s),
+ *   T = softmax(u_t);
+ *   beta == 0:   loss_n = KL(T || S)              (forward KL)
+ *   beta == 1:   loss_n = KL(S || T)              (reverse KL, the OPD objective)
+ *   0 < beta < 1: loss_n = beta KL(T || M) + (1 - beta) KL(S || M),
+ *                 M = (1 - beta) S + beta T       (generalized JSD)
+ *   loss_mean = sum over rows with label != ignore_index of loss_n / N_v
+ *   (a per-token mean; 0 when N_v == 0).
+ * The teacher is frozen: the backward returns dL/dh_s and dL/dW_s only.
+ *
+ * Layouts: h_s [n_tokens, d_s], h_t [n_tokens, d_t] row-major (bf16 or fp32, see
+ * nb_kl_shape.h_dtype); W_s [vocab, d_s], W_t [vocab, d_t] row-major bf16; labels
+ * [n_tokens] int64; every per-token output [n_tokens] fp32; dh_s [n_tokens, d_s] fp32;
+ * dW_s [vocab, d_s] fp32. Row n of h_s, h_t and labels is one position (no shift).
+ *
+ * Requirements (NB_ERR_INVALID_ARG otherwise): d_s and d_t multiples of 8; h_*, W_*
+ * and the workspace 16-byte aligned; 0 <= beta <= 1; tau > 0 and finite;
+ * workspace_bytes >= nb_kl_workspace_size(shape, beta). n_tokens may be 0.
+ *
+ * Errors: invalid arguments are reported synchronously by the return value and launch
+ * nothing. Device-side failures (a bounded wait that ran out) are written to a status
+ * word inside the workspace; nb_kl_device_status() reads it. Every forward/backward call
+ * clears that word when it starts.
+ */
+#ifndef NB_KL_H
+#define NB_KL_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define NB_KL_API __attribute__((visibility("default")))
+#else
+#define NB_KL_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum nb_status {
+  NB_OK = 0,
+  NB_ERR_INVALID_ARG = -1,  /* null/misaligned pointer, bad size, beta or tau out of range */
+  NB_ERR_UNSUPPORTED = -2,  /* no sm_100 device, or a size beyond what the kernels index */
+  NB_ERR_WORKSPACE = -3,    /* workspace smaller than nb_kl_workspace_size() */
+  NB_ERR_CUDA = -4,         /* a CUDA runtime / driver call failed */
+  NB_ERR_TIMEOUT = -5       /* a bounded device-side wait ran out (device status word) */
+} nb_status;
+
+typedef enum nb_dtype { NB_BF16 = 0, NB_F32 = 1 } nb_dtype;
+
+typedef struct nb_kl_shape {
+  int64_t n_tokens;     /* N = B * T rows of h_s, h_t, labels */
+  int64_t vocab;        /* V */
+  int64_t d_s;          /* student hidden width */
+  int64_t d_t;          /* teacher hidden width (or the rank of a compressed teacher code) */
+  int32_t h_dtype;      /* nb_dtype of h_s and h_t; W_s and W_t are always bf16 */
+  int32_t reserved;     /* must be 0 */
+  int64_t ignore_index; /* label of masked positions, normally -100 */
+  int64_t chunk_v;      /* backward vocabulary chunk (multiple of 128); 0 = library default */
+} nb_kl_shape;
+
+/* Bytes of scratch the calls need for this shape: O(n_tokens * (d_s + d_t + chunk_v))
+ * plus O(n_tokens * vocab / 2048) floats of split-V state — never O(n_tokens * vocab).
+ * Returns 0 for an invalid shape. */
+NB_KL_API size_t nb_kl_workspace_size(const nb_kl_shape* shape, float beta);
+
+/* Forward ("Nitrobrew 的两个动作": block GEMMs + online log-sum-exp + KL numerator).
+ * Outputs (device, caller-owned): loss_tok, lse_s, lse_t, aux [n_tokens] fp32 —
+ * lse_* are natural-log LSEs of the tempered logits u = z / tau; aux is the per-token KL
+ * for beta in {0, 1} and KL(S || M) for 0 < beta < 1 (the backward needs it); masked rows
+ * get 0 in all four. loss_mean: one fp32; n_valid: one int64 (N_v). */
+NB_KL_API nb_status nb_kl_forward(const nb_kl_shape* shape, const void* h_s, const void* W_s, const void* h_t,
+                        const void* W_t, const int64_t* labels, float beta, float tau, float* loss_tok,
+                        float* lse_s, float* lse_t, float* aux, float* loss_mean, int64_t* n_valid,
+                        void* workspace, size_t workspace_bytes, void* stream);
+
+/* Backward ("仓库实现": recompute the logit blocks; gradients reach h_s and W_s only).
+ * Inputs lse_s, lse_t, aux are the forward's outputs for the same arguments; grad_out is
+ * one fp32 on the device (dOut/dloss_mean). Writes dh_s [n_tokens, d_s] (masked rows 0)
+ * and dW_s [vocab, d_s]: overwritten, or added to when accumulate_dW != 0. */
+NB_KL_API nb_status nb_kl_backward(const nb_kl_shape* shape, const void* h_s, const void* W_s, const void* h_t,
+                         const void* W_t, const int64_t* labels, float beta, float tau, const float* lse_s,
+                         const float* lse_t, const float* aux, const float* grad_out, float* dh_s, float* dW_s,
+                         int accumulate_dW, void* workspace, size_t workspace_bytes, void* stream);
+
+/* Static text for a status code. */
+NB_KL_API const char* nb_kl_status_string(nb_status status);
+
+/* Synchronises `stream`, then returns the device status word of `workspace`
+ * (NB_OK, or NB_ERR_TIMEOUT after a bounded wait ran out), or NB_ERR_CUDA. */
+NB_KL_API nb_status nb_kl_device_status(void* workspace, void* stream);
+
+/* ---- test hooks (no counterpart on the pages) ---------------------------------------- */
+
+/* C[M, N] = sum_k A[m, k] B[n, k] in fp32 with the library's tcgen05 GEMM. A is stored
+ * row-major as [M, K] (a_mn_major = 0) or [K, M] (a_mn_major = 1); B as [N, K]
+ * (b_mn_major = 0) or [K, N] (b_mn_major = 1); bf16, 16-byte aligned, leading
+ * dimensions multiples of 8. workspace needs 256 bytes (status word). */
+NB_KL_API nb_status nb_kl_debug_gemm(const void* A, int a_mn_major, const void* B, int b_mn_major, int64_t M, int64_t N,
+                           int64_t K, float* C, void* workspace, void* stream);
+
+/* Launches a kernel whose mbarrier wait can never complete, bounded by limit_ns, so that
+ * the timeout path can be exercised without hanging the GPU. Afterwards
+ * nb_kl_device_status(workspace) reports NB_ERR_TIMEOUT. workspace: 256 bytes. */
+NB_KL_API nb_status nb_kl_debug_wait_timeout(void* workspace, uint64_t limit_ns, void* stream);
+
+/* Number of kernel launches the last forward / backward call on this thread made. */
+NB_KL_API int nb_kl_last_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* NB_KL_H */

@@ -164,12 +164,14 @@ def forward(h_s, W_s, h_t, W_t, labels, beta: float, tau: float, *,
 
 def backward(h_s, W_s, h_t, W_t, labels, beta: float, tau: float, *, grad_out: float = 1.0,
              dW_init: Optional[np.ndarray] = None, rows: Optional[Sequence[int]] = None,
-             want_dW: bool = True, ignore_index: int = IGNORE_INDEX, row_block: int = 256) -> dict:
+             want_dW: bool = True, dW_rows: Optional[Sequence[int]] = None,
+             ignore_index: int = IGNORE_INDEX, row_block: int = 256) -> dict:
     """Gradients of ``grad_out * mean_loss`` w.r.t. h_s and W_s (the teacher is frozen).
 
     ``G[n, v] = grad_out / (N_v * tau) * d loss_n / d u_s[n, v]`` on valid rows,
     ``dh_s = G @ W_s`` and ``dW_s = G^T @ h_s`` (plus ``dW_init`` when given).
     With ``rows`` only those rows of ``dh_s`` are produced and ``dW_s`` is left out.
+    With ``dW_rows`` only those vocabulary rows of ``dW_s`` are produced (in that order).
     """
     _check(beta, tau)
     labels = np.asarray(labels)
@@ -181,8 +183,12 @@ def backward(h_s, W_s, h_t, W_t, labels, beta: float, tau: float, *, grad_out: f
     want_dW = want_dW and rows is None
     dh = np.zeros((N, d_s))
     dW = None
+    sel = None if dW_rows is None else np.asarray(dW_rows, dtype=np.int64)
     if want_dW:
-        dW = np.zeros((W_s.shape[0], d_s)) if dW_init is None else np.array(dW_init, dtype=np.float64)
+        if sel is None:
+            dW = np.zeros((W_s.shape[0], d_s)) if dW_init is None else np.array(dW_init, dtype=np.float64)
+        else:
+            dW = np.zeros((len(sel), d_s)) if dW_init is None else np.array(dW_init[sel], dtype=np.float64)
     if n_valid == 0:
         return {"dh_s": dh, "dW_s": dW}
     scale = grad_out / (n_valid * tau)
@@ -194,6 +200,8 @@ def backward(h_s, W_s, h_t, W_t, labels, beta: float, tau: float, *, grad_out: f
         for v0 in range(0, W_s.shape[0], _V_BLOCK):
             v1 = min(W_s.shape[0], v0 + _V_BLOCK)
             dh[r] += G[:, v0:v1] @ _to_f64(W_s[v0:v1])
-            if want_dW:
+            if want_dW and sel is None:
                 dW[v0:v1] += G[:, v0:v1].T @ _to_f64(h_s[r])
+        if want_dW and sel is not None:
+            dW += G[:, sel].T @ _to_f64(h_s[r])
     return {"dh_s": dh, "dW_s": dW}

@@ -366,3 +366,14 @@ def test_reverse_kl_gradient_blows_up_as_teacher_prob_vanishes():
         norms.append(np.linalg.norm(g))
     assert all(b > a for a, b in zip(norms, norms[1:]))
     assert norms[-1] > 3 * norms[0]
+
+
+def test_dW_rows_selection_matches_full():
+    rng = np.random.default_rng(16)
+    h_s, W_s, h_t, W_t = rand_problem(rng, 7, 30, 5, 6, scale=2.0)
+    lab = np.array([1, -100, 3, 4, 5, 6, -100])
+    init = rng.standard_normal((30, 5))
+    full = oracle.backward(h_s, W_s, h_t, W_t, lab, 0.4, 1.3, dW_init=init)["dW_s"]
+    sel = [29, 0, 7, 7, 15]
+    part = oracle.backward(h_s, W_s, h_t, W_t, lab, 0.4, 1.3, dW_init=init, dW_rows=sel)["dW_s"]
+    np.testing.assert_allclose(part, full[sel], rtol=1e-13, atol=1e-16)
