@@ -1,0 +1,414 @@
+"""Benchmark: fused forward + backward of the full-vocabulary distillation loss.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl library|reference]
+
+One step = nb_kl_forward + nb_kl_backward over one batch of the workload (every step of
+the hot path: compaction, both block GEMMs with the online LSE/KL epilogue, split-V merge,
+[JSD second sweep], masked mean, recompute sweep, dh_s and dW_s GEMMs). Inputs are resident
+in HBM when the timed region starts; the unembeddings (>= 1 GB per step) are larger than
+L2, so no explicit flush is needed between steps. The timed region is bracketed by a
+barrier and a device synchronisation and timed with CUDA events on the launching stream;
+with N > 1 every rank runs its own replica (no data-path collective) and the time is the
+maximum over ranks.
+
+Prints one JSON line. `value` is whole-job tokens/s (all B*T positions of every rank);
+`e2e` repeats the measurement through the public API with the step's inputs copied from
+pinned host memory and the loss read back each step; `roofline` describes the dominant
+kernel; `cpu_baseline` times the fp64 oracle on a bounded sample on this host.
+"""
+
+from __future__ import annotations
+
+import argparse
+import ctypes
+import hashlib
+import json
+import math
+import os
+import re
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "distill-loss tokens/sec (fwd+bwd) at V=151936; % of bf16 tensor peak"
+DATASHEET_BF16_TFLOPS = 2250.0
+FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+DEFAULT_WORKLOAD = "opd_0p6b_4b"
+
+
+# ----------------------------------------------------------------------------- helpers
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK), "fallback"
+
+
+def algorithmic_flops(w, n_valid):
+    """FLOPs of the method on valid rows: forward sweep, [JSD second sweep], recompute sweep,
+    dh_s and dW_s products."""
+    sweep = 2.0 * n_valid * w.V * (w.d_s + w.d_t)
+    jsd = 0.0 < w.beta < 1.0
+    return {
+        "sweep_fwd": sweep,
+        "sweep_jsd": sweep if jsd else 0.0,
+        "sweep_grad": sweep,
+        "gemm_bwd": 4.0 * n_valid * w.V * w.d_s,
+    }
+
+
+def kernel_source_sha():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "full_vocab_kl_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(kernel: str, workload: str):
+    """Per-launch DRAM bytes from a committed ncu summary, if it matches the current source."""
+    p = os.path.join(ROOT, "profiles", f"{kernel}_{workload}.md")
+    if not os.path.exists(p):
+        return None
+    txt = open(p).read()
+    m_sha = re.search(r"kernel_source_sha:\s*([0-9a-f]+)", txt)
+    m_tr = re.search(r"dram_bytes_per_launch:\s*([0-9.eE+]+)", txt)
+    if not m_sha or not m_tr or m_sha.group(1) != kernel_source_sha():
+        return None
+    return float(m_tr.group(1))
+
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.proc = None
+        self.gpu = gpu_index
+        self.path = f"/tmp/nbkl_clocks_{os.getpid()}.csv"
+
+    def start(self):
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=self.f, stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.15)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.f.close()
+        sm, smax, reasons, power = [], [], set(), []
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+                power.append(float(parts[3]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        os.remove(self.path)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        busy = [s for s in sm if s > 0.5 * max(sm)] or sm
+        return {"sm_mhz": float(np.median(busy)), "sm_max_mhz": float(max(smax)), "reasons": sorted(reasons),
+                "samples": len(sm), "power_w_max": float(max(power)) if power else None}
+
+
+# ----------------------------------------------------------------------------- oracle timing
+def oracle_sample_run(x, positions):
+    """One oracle pass (forward + backward incl. dW_s) over the given positions only."""
+    import oracle
+    sub = np.full_like(x.labels, -100)
+    sub[positions] = x.labels[positions]
+    oracle.forward(x.h_s, x.W_s, x.h_t, x.W_t, sub, x.beta, x.tau)
+    oracle.backward(x.h_s, x.W_s, x.h_t, x.W_t, sub, x.beta, x.tau, grad_out=x.grad_out)
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads") for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:  # pragma: no cover
+        pass
+    return len(os.sched_getaffinity(0))
+
+
+def cpu_baseline(x, budget_s=15.0):
+    rng = np.random.default_rng(7)
+    N = x.labels.shape[0]
+    t0 = time.perf_counter()
+    first = np.sort(rng.choice(N, size=64, replace=False))
+    oracle_sample_run(x, first)
+    t1 = time.perf_counter() - t0
+    n = int(min(N, max(64, 64 * (budget_s / max(t1, 1e-3)))))
+    pos = np.sort(rng.choice(N, size=n, replace=False))
+    t0 = time.perf_counter()
+    oracle_sample_run(x, pos)
+    dt = time.perf_counter() - t0
+    nv = int((x.labels[pos] != -100).sum())
+    return {"value": n / dt, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+            "sample": f"{n} of {N} positions ({nv} valid) of workload {x.workload.name}, "
+                      f"forward + backward incl. dW_s, fp64 NumPy, {dt:.1f} s"}
+
+
+# ----------------------------------------------------------------------------- reference arm
+def run_reference(args):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return 0
+    from synthetic import make_inputs
+    x = make_inputs(args.workload)
+    N = x.labels.shape[0]
+    rng = np.random.default_rng(11)
+    budget = 150.0 / max(1, args.steps + args.warmup)
+    t0 = time.perf_counter()
+    oracle_sample_run(x, np.sort(rng.choice(N, size=32, replace=False)))
+    per_pos = (time.perf_counter() - t0) / 32
+    n = int(max(16, min(N, budget / max(per_pos, 1e-6))))
+    for _ in range(args.warmup):
+        oracle_sample_run(x, np.sort(rng.choice(N, size=n, replace=False)))
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle_sample_run(x, np.sort(rng.choice(N, size=n, replace=False)))
+    dt = time.perf_counter() - t0
+    value = n * args.steps / dt
+    w = x.workload
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": workload_config(w, int((x.labels != -100).sum()), 1),
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+                         "sample": f"{n} random positions of {N} per step, forward + backward incl. dW_s"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def workload_config(w, n_valid, world):
+    return {"workload": w.name, "global_batch": w.B * world, "seq_len": w.T, "tokens_per_rank": w.N,
+            "valid_tokens_per_rank": n_valid, "vocab": w.V, "d_s": w.d_s, "d_t": w.d_t, "beta": w.beta,
+            "tau": w.tau, "parallelism": f"replicas{world}" if world > 1 else "single",
+            "l2": "inputs larger than L2 (unembeddings >= 1 GB per step), no flush"}
+
+
+# ----------------------------------------------------------------------------- library arm
+def run_library(args):
+    import torch
+    import torch.distributed as dist
+
+    import full_vocab_kl_b200 as nb
+    from full_vocab_kl_b200 import _abi
+    from synthetic import make_inputs
+
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+
+    x = make_inputs(args.workload)
+    w = x.workload
+    n_valid = int((x.labels != -100).sum())
+
+    def to_dev(a):
+        if a.dtype == np.uint16:
+            return torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(dev)
+        return torch.from_numpy(a).to(dev)
+
+    h_s, h_t, W_s, W_t = (to_dev(getattr(x, k)) for k in ("h_s", "h_t", "W_s", "W_t"))
+    labels = torch.from_numpy(x.labels).to(dev)
+    shape = nb.make_shape(h_s, W_s, h_t, W_t, labels)
+    ws_bytes = nb.workspace_bytes(shape, w.beta)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    N = labels.shape[0]
+    f32 = dict(dtype=torch.float32, device=dev)
+    out = {"loss_tok": torch.empty(N, **f32), "lse_s": torch.empty(N, **f32), "lse_t": torch.empty(N, **f32),
+           "aux": torch.empty(N, **f32), "loss_mean": torch.empty((), **f32),
+           "n_valid": torch.empty((), dtype=torch.int64, device=dev)}
+    dh = torch.empty((N, w.d_s), **f32)
+    dW = torch.zeros((w.V, w.d_s), **f32) if w.accumulate_dW else torch.empty((w.V, w.d_s), **f32)
+    grad_out = torch.ones((), **f32)
+    lib = _abi.lib()
+
+    def step(hs, ht, lab):
+        nb.kl_forward(hs, W_s, ht, W_t, lab, w.beta, w.tau, workspace=ws, out=out)
+        n1 = lib.nb_kl_last_launch_count()
+        nb.kl_backward(hs, W_s, ht, W_t, lab, w.beta, w.tau, out["lse_s"], out["lse_t"], out["aux"], grad_out,
+                       dh_s=dh, dW_s=dW, accumulate_dW=w.accumulate_dW, workspace=ws)
+        return n1 + lib.nb_kl_last_launch_count()
+
+    stream = torch.cuda.current_stream(dev)
+    for _ in range(args.warmup):
+        step(h_s, h_t, labels)
+    mem0 = torch.cuda.memory_allocated(dev)
+    torch.cuda.reset_peak_memory_stats(dev)
+
+    # ---- device-timed region
+    clocks = ClockSampler(local)
+    if rank == 0:
+        clocks.start()
+    lib.nb_kl_timing_enable(1)
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    launches = 0
+    for _ in range(args.steps):
+        launches += step(h_s, h_t, labels)
+    e1.record(stream)
+    barrier()
+    lib.nb_kl_timing_enable(0)
+    ms_arr = (ctypes.c_double * 5)()
+    cnt_arr = (ctypes.c_int * 5)()
+    lib.nb_kl_timing_read(ctypes.cast(ms_arr, ctypes.c_void_p), ctypes.cast(cnt_arr, ctypes.c_void_p), 5)
+    clk = clocks.stop() if rank == 0 else None
+    ms = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    peak_extra = torch.cuda.max_memory_allocated(dev) - mem0
+
+    # ---- end-to-end through the public API with host buffers
+    pin = {}
+    for k, t in (("h_s", h_s), ("h_t", h_t), ("labels", labels)):
+        pin[k] = torch.empty(t.shape, dtype=t.dtype, pin_memory=True)
+        pin[k].copy_(t)
+    loss_host = torch.empty((2,), dtype=torch.float64, pin_memory=True)
+    hs_d, ht_d, lab_d = torch.empty_like(h_s), torch.empty_like(h_t), torch.empty_like(labels)
+    h2d = sum(t.numel() * t.element_size() for t in pin.values())
+    d2h = out["loss_mean"].element_size() + out["n_valid"].element_size()
+    e2e_steps = max(3, min(args.steps, 20))
+
+    def e2e_step():
+        hs_d.copy_(pin["h_s"], non_blocking=True)
+        ht_d.copy_(pin["h_t"], non_blocking=True)
+        lab_d.copy_(pin["labels"], non_blocking=True)
+        step(hs_d, ht_d, lab_d)
+        loss_host[0].copy_(out["loss_mean"], non_blocking=True)
+        loss_host[1].copy_(out["n_valid"], non_blocking=True)
+        stream.synchronize()
+        return float(loss_host[0])
+
+    e2e_step()
+    barrier()
+    e2, e3 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e2.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e3.record(stream)
+    barrier()
+    ms_e2e = e2.elapsed_time(e3)
+    if world > 1:
+        t = torch.tensor([ms_e2e], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_e2e = float(t.item())
+
+    result = None
+    if rank == 0:
+        ms_step = ms / args.steps
+        tokens = N * world
+        value = tokens / (ms_step * 1e-3)
+        flops = algorithmic_flops(w, n_valid)
+        step_flops = sum(flops.values())
+        tflops = step_flops / (ms_step * 1e-3) / 1e12
+        peaks, peak_src = measured_peaks()
+        cats = _abi.KERNEL_CATEGORIES
+        kms = {c: ms_arr[i] / args.steps for i, c in enumerate(cats)}
+        kcount = {c: cnt_arr[i] / args.steps for i, c in enumerate(cats)}
+        dom = max(("sweep_fwd", "sweep_jsd", "sweep_grad", "gemm_bwd"), key=lambda c: kms[c])
+        per_launch_ms = kms[dom] / max(kcount[dom], 1)
+        per_launch_flops = flops[dom] / max(kcount[dom], 1)
+        achieved = per_launch_flops / (per_launch_ms * 1e-3) / 1e12
+        peak = peaks.get("bf16_tflops_sustained", FALLBACK["bf16_tflops_sustained"])
+        traffic = profiled_traffic(dom, w.name)
+        result = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded; shapes of the workload)",
+            "config": workload_config(w, n_valid, world),
+            "tflops": tflops, "pct_bf16_peak_datasheet": 100.0 * tflops / DATASHEET_BF16_TFLOPS,
+            "pct_bf16_peak_measured": 100.0 * tflops / peaks.get("bf16_tflops", FALLBACK["bf16_tflops"]),
+            "roofline": {"bound": "tensor", "kernel": dom, "achieved": achieved, "peak": peak,
+                         "peak_source": f"{peak_src} bf16_tflops_sustained", "unit": "TFLOP/s",
+                         "frac": achieved / peak, "traffic": traffic,
+                         "algorithmic_flops_per_launch": per_launch_flops, "launch_ms": per_launch_ms},
+            "kernel_ms_per_step": kms, "kernel_launches_per_step": kcount,
+            "e2e": {"value": tokens / (ms_e2e / e2e_steps * 1e-3), "unit": "tokens/s",
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps},
+            "gpu_launches": launches,
+            "clocks": clk,
+            "scratch_bytes": ws_bytes, "peak_extra_alloc_bytes": int(peak_extra),
+        }
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0 and not args.no_cpu_baseline:
+        result["cpu_baseline"] = cpu_baseline(x)
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD,
+                    help="a workload name (synthetic.WORKLOADS) or a profiling-size one (synthetic.PROFILE_WORKLOADS)")
+    ap.add_argument("--impl", default="library", choices=["library", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_library(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

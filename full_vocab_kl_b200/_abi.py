@@ -37,7 +37,11 @@ SIGNATURES = {
                                  c_void_p]),
     "nb_kl_debug_wait_timeout": (c_int, [c_void_p, c_uint64, c_void_p]),
     "nb_kl_last_launch_count": (c_int, []),
+    "nb_kl_timing_enable": (None, [c_int]),
+    "nb_kl_timing_read": (c_int, [c_void_p, c_void_p, c_int]),
 }
+
+KERNEL_CATEGORIES = ("sweep_fwd", "sweep_jsd", "sweep_grad", "gemm_bwd", "rowops")
 
 
 class Shape(ctypes.Structure):

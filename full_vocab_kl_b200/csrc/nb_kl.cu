@@ -14,6 +14,7 @@
 #include <cstdint>
 #include <cstring>
 #include <mutex>
+#include <vector>
 
 #include "../../include/nb_kl.h"
 #include "common.cuh"
@@ -31,6 +32,29 @@ constexpr int64_t kDefaultChunkV = 8192;
 constexpr size_t kCtrlBytes = 256;
 
 thread_local int g_launches = 0;
+
+// Opt-in per-kernel timing: events recorded on the launching stream around each launch.
+struct TimingRec {
+  int cat;
+  cudaEvent_t a, b;
+};
+struct Timing {
+  bool on = false;
+  std::vector<TimingRec> recs;
+  std::vector<cudaEvent_t> pool;
+  cudaEvent_t get() {
+    if (!pool.empty()) {
+      cudaEvent_t e = pool.back();
+      pool.pop_back();
+      return e;
+    }
+    cudaEvent_t e = nullptr;
+    cudaEventCreate(&e);
+    return e;
+  }
+};
+thread_local Timing g_timing;
+thread_local int g_cat = NB_KL_KERNEL_ROWOPS;
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 int64_t round_up(int64_t x, int64_t m) { return (x + m - 1) / m * m; }
@@ -160,9 +184,23 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 
 
 template <typename K, typename... Args>
 void launch(K kernel, dim3 grid, dim3 block, size_t smem, cudaStream_t st, Args... args) {
+  TimingRec r{g_cat, nullptr, nullptr};
+  if (g_timing.on) {
+    r.a = g_timing.get();
+    r.b = g_timing.get();
+    cudaEventRecord(r.a, st);
+  }
   kernel<<<grid, block, smem, st>>>(args...);
   ++g_launches;
+  if (g_timing.on) {
+    cudaEventRecord(r.b, st);
+    g_timing.recs.push_back(r);
+  }
+  g_cat = NB_KL_KERNEL_ROWOPS;
 }
+
+// the next launch belongs to category `c`
+void next_cat(int c) { g_cat = c; }
 
 nb_status check_launch() { return cudaGetLastError() == cudaSuccess ? NB_OK : NB_ERR_CUDA; }
 
@@ -253,6 +291,7 @@ int sweep_grid(const DevInfo& dev, const Layout& L, const SweepArgs& a) {
 
 template <int MODE>
 void launch_sweep(const DevInfo& dev, const Layout& L, const SweepMaps& m, const SweepArgs& a, cudaStream_t st) {
+  next_cat(MODE <= kStateT ? NB_KL_KERNEL_SWEEP_FWD : MODE == kJsd ? NB_KL_KERNEL_SWEEP_JSD : NB_KL_KERNEL_SWEEP_GRAD);
   launch(sweep_kernel<MODE>, dim3(sweep_grid(dev, L, a)), dim3(kThreads), size_t(kSmemBytes), st, m, a);
 }
 
@@ -295,6 +334,30 @@ const char* nb_kl_status_string(nb_status s) {
 }
 
 int nb_kl_last_launch_count(void) { return g_launches; }
+
+void nb_kl_timing_enable(int on) { g_timing.on = on != 0; }
+
+int nb_kl_timing_read(double* ms, int* launches, int ncat) {
+  if (ncat < 0) return -1;
+  for (int i = 0; i < ncat; ++i) {
+    if (ms) ms[i] = 0.0;
+    if (launches) launches[i] = 0;
+  }
+  int n = 0;
+  for (const TimingRec& r : g_timing.recs) {
+    float t = 0.f;
+    if (cudaEventSynchronize(r.b) == cudaSuccess && cudaEventElapsedTime(&t, r.a, r.b) == cudaSuccess &&
+        r.cat >= 0 && r.cat < ncat) {
+      if (ms) ms[r.cat] += t;
+      if (launches) launches[r.cat] += 1;
+    }
+    g_timing.pool.push_back(r.a);
+    g_timing.pool.push_back(r.b);
+    ++n;
+  }
+  g_timing.recs.clear();
+  return n;
+}
 
 nb_status nb_kl_device_status(void* workspace, void* stream) {
   if (!workspace) return NB_ERR_INVALID_ARG;
@@ -445,6 +508,7 @@ nb_status nb_kl_backward(const nb_kl_shape* shape, const void* h_s, const void* 
     dw.M = int(v1 - v0);
     dw.out = dW_s + v0 * L.d_s;
     const int tiles = n_tt_max * n_dt + int((v1 - v0 + kBlockM - 1) / kBlockM) * n_dt;
+    next_cat(NB_KL_KERNEL_GEMM_BWD);
     launch(gemm_kernel, dim3(std::max(1, std::min(dev.sms, tiles))), dim3(kThreads), size_t(kSmemBytes), st, gm, g);
   }
   return check_launch();

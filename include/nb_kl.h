@@ -120,6 +120,27 @@ NB_KL_API nb_status nb_kl_debug_wait_timeout(void* workspace, uint64_t limit_ns,
 /* Number of kernel launches the last forward / backward call on this thread made. */
 NB_KL_API int nb_kl_last_launch_count(void);
 
+/* ---- measurement hooks (no counterpart on the pages) --------------------------------- */
+
+/* Kernel categories of the timing hook. */
+enum {
+  NB_KL_KERNEL_SWEEP_FWD = 0,   /* forward vocabulary sweep (block GEMMs + online LSE/KL) */
+  NB_KL_KERNEL_SWEEP_JSD = 1,   /* second forward sweep of the JSD */
+  NB_KL_KERNEL_SWEEP_GRAD = 2,  /* backward recompute sweep writing the gradient chunk */
+  NB_KL_KERNEL_GEMM_BWD = 3,    /* backward dh_s / dW_s GEMMs */
+  NB_KL_KERNEL_ROWOPS = 4,      /* compaction, merges, mean */
+  NB_KL_KERNEL_CATEGORIES = 5
+};
+
+/* Per calling thread: when on, every launch is bracketed by two CUDA events recorded on
+ * its stream (no synchronisation is added). Off by default. */
+NB_KL_API void nb_kl_timing_enable(int on);
+
+/* Waits for the recorded events, writes the summed milliseconds and launch counts per
+ * category into ms[ncat] / launches[ncat] (either may be NULL), clears the record and
+ * returns the number of launches read. */
+NB_KL_API int nb_kl_timing_read(double* ms, int* launches, int ncat);
+
 #ifdef __cplusplus
 }
 #endif

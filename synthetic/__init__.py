@@ -9,6 +9,7 @@ from .workloads import (  # noqa: F401
     IGNORE_INDEX,
     WORKLOADS,
     Inputs,
+    PROFILE_WORKLOADS,
     Workload,
     bf16_bits_to_f32,
     f32_to_bf16_bits,

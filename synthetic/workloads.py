@@ -99,6 +99,16 @@ WORKLOADS = {
 }
 
 
+# Same widths and statistics as a named workload but fewer tokens and a smaller vocabulary,
+# so that a detailed profiler capture of one kernel stays small (inputs still exceed L2).
+PROFILE_WORKLOADS = {
+    "opd_0p6b_4b_prof": Workload(
+        "opd_0p6b_4b_prof", 1, 2048, 1024, 2560, 32768, 1.0, 1.0, 3.0,
+        teacher="correlated", mask="prefix", masked_per_seq=819,
+        description="profiling size of opd_0p6b_4b: 2048 tokens, V 32768"),
+}
+
+
 # ----------------------------------------------------------------------------------------
 # bf16 byte handling
 # ----------------------------------------------------------------------------------------
@@ -233,7 +243,10 @@ def _signed_embedding(seed: int, d_s: int, d_t: int):
 
 def make_inputs(name_or_workload, seed: int = 0) -> Inputs:
     """Generate the seeded inputs of a named workload (or a custom :class:`Workload`)."""
-    w = WORKLOADS[name_or_workload] if isinstance(name_or_workload, str) else name_or_workload
+    if isinstance(name_or_workload, str):
+        w = WORKLOADS.get(name_or_workload) or PROFILE_WORKLOADS[name_or_workload]
+    else:
+        w = name_or_workload
     N, d_s, d_t, V = w.N, w.d_s, w.d_t, w.V
     sd_s, sd_t = w.w_std / math.sqrt(d_s), w.w_std / math.sqrt(d_t)
 
