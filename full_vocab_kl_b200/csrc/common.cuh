@@ -9,24 +9,35 @@
 
 namespace nbkl {
 
-// One CTA owns a 128-token x 128-column output tile; K advances 64 bf16 (one 128-byte
-// swizzle row) per pipeline stage.
+// One CTA owns a 128-token x 256-column output tile (the MMA instruction is 128 x 256 x 16:
+// with N = 128 the tensor pipe stays busy for the same time and delivers half the work);
+// K advances 64 bf16 (one 128-byte swizzle row) per pipeline stage.
 constexpr int kBlockM = 128;
-constexpr int kBlockN = 128;
+constexpr int kBlockN = 256;
 constexpr int kBlockK = 64;
-constexpr int kStages = 6;
-constexpr int kTileBytes = kBlockM * kBlockK * 2;      // 16 KB per operand per stage
-constexpr int kStageBytes = 2 * kTileBytes;            // A + B
-constexpr int kThreads = 192;                          // TMA warp, MMA warp, 4 epilogue warps
-constexpr int kEpiThreads = 128;
+constexpr int kStages = 4;
+constexpr int kATileBytes = kBlockM * kBlockK * 2;     // 16 KB
+constexpr int kBTileBytes = kBlockN * kBlockK * 2;     // 32 KB
+constexpr int kStageBytes = kATileBytes + kBTileBytes; // 48 KB
+constexpr int kEpiWarps = 8;                           // two warps per TMEM lane quarter
+constexpr int kEpiWarp0 = 4;                           // epilogue = warpgroups 1 and 2
+constexpr int kEpiThreads = kEpiWarps * 32;
+constexpr int kThreads = 128 + kEpiThreads;            // warpgroup 0: TMA warp, MMA warp, 2 idle
+// Register split: warpgroup 0 gives registers back, the epilogue warpgroups take them.
+// 128 * kRegsCtl + 256 * kRegsEpi must not exceed 384 * (registers at launch = 168).
+constexpr int kRegsLaunch = 168;
+constexpr int kRegsCtl = 56;
+constexpr int kRegsEpi = 224;
+static_assert(128 * kRegsCtl + kEpiThreads * kRegsEpi <= kThreads * kRegsLaunch, "register split");
+constexpr int kHalfN = kBlockN / 2;                    // columns per epilogue thread per tile
 constexpr int kSmemBytes = kStages * kStageBytes + 1024 /*align*/ + 256 /*barriers*/;
 
 constexpr float kLn2 = 0.69314718055994530942f;
 constexpr float kLog2e = 1.44269504088896340736f;
 constexpr float kNegBig = -1.0e30f;  // finite "minus infinity" for masked columns
 
-// Idesc for the 128 x 128 tiles used everywhere.
-constexpr uint32_t kIdescKK = make_idesc(128, 128, 0, 0);
+// Idesc of the sweep's 128 x 256 K-major x K-major products.
+constexpr uint32_t kIdescKK = make_idesc(kBlockM, kBlockN, 0, 0);
 
 __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
   return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
@@ -48,6 +59,7 @@ struct SweepMaps {
 };
 
 struct SweepArgs {
+  int teacher_first;      // MMA order / epilogue order: the model with the larger K goes first
   int V;                  // vocabulary size
   int v_begin, v_end;     // vocabulary columns covered by this launch
   int nkb_s, nkb_t;       // K blocks of the A operands (student, teacher)
@@ -55,7 +67,8 @@ struct SweepArgs {
   int tiles_per_unit;     // vocabulary tiles per work unit (one split of the LSE state)
   float scale;            // log2(e) / tau: base-2 tempered logits x = z * scale
   float beta, lg2_1mb, lg2_b;
-  float* out;             // state [5][split][ld] or JSD partial sums [2][split][ld]
+  float* out;             // state [5][split][ld] or JSD partial sums [2][split][ld]; split =
+                          // 2 * unit + column half
   long long field_stride; // elements between fields of `out`
   int ld;                 // rows per split in `out`
   const float* row_l2s;   // per compacted row: base-2 LSE of the student (pass 2, backward)

@@ -9,8 +9,8 @@
 // G^T, W_s[chunk] (as K x N) and h_s (as K x N) are read MN-major straight from their
 // row-major buffers through 64 x 64 TMA boxes, so nothing is transposed in memory.
 //
-// Same warp roles as the sweep: warp 0 TMA, warp 1 MMA (one 128-column fp32 accumulator,
-// double-buffered in TMEM), warps 2-5 write one output row per thread.
+// Same warp roles as the sweep: warp 0 TMA, warp 1 MMA (one 128 x 256 fp32 accumulator,
+// double-buffered in TMEM), warps 4-11 write one output row half (128 columns) per thread.
 #pragma once
 
 #include "common.cuh"
@@ -54,15 +54,14 @@ __device__ __forceinline__ int total_tiles(const GemmArgs& p, int nv) {
   return t;
 }
 
-// K-major operand: one 128-row x 64-column box. MN-major operand: two 64 x 64 boxes
-// (MN columns mn0..mn0+63 and mn0+64..mn0+127) stacked 8 KB apart.
+// K-major operand: one (rows x 64) box. MN-major operand: (rows / 64) boxes of 64 x 64
+// (64 MN columns each) stacked 8 KB apart.
 __device__ __forceinline__ void load_operand(uint32_t dst, const CUtensorMap* map, uint32_t bar, int mn_major,
-                                             int mn0, int kcoord) {
+                                             int mn0, int kcoord, int rows) {
   if (!mn_major) {
     tma_load_2d(dst, map, bar, kcoord, mn0);
   } else {
-    tma_load_2d(dst, map, bar, mn0, kcoord);
-    tma_load_2d(dst + kTileBytes / 2, map, bar, mn0 + 64, kcoord);
+    for (int i = 0; i < rows / 64; ++i) tma_load_2d(dst + i * 8192, map, bar, mn0 + 64 * i, kcoord);
   }
 }
 
@@ -70,7 +69,7 @@ __device__ __forceinline__ uint64_t operand_desc(uint32_t saddr, int mn_major, i
   // K-major: 8-row groups 1024 B apart, K step of 16 elements = 32 B inside the swizzle row.
   // MN-major: 64-wide MN atoms 8 KB apart (LBO), 8-row K groups 1024 B apart (SBO),
   // K step of 16 rows = 2048 B.
-  return mn_major ? make_sdesc(saddr + j * 2048, kTileBytes / 2, 1024) : make_sdesc(saddr + j * 32, 16, 1024);
+  return mn_major ? make_sdesc(saddr + j * 2048, 8192, 1024) : make_sdesc(saddr + j * 32, 16, 1024);
 }
 
 __device__ __forceinline__ void gemm_producer(const GemmMaps& maps, const GemmArgs& p, int nv, const SweepSmem& s,
@@ -89,26 +88,17 @@ __device__ __forceinline__ void gemm_producer(const GemmMaps& maps, const GemmAr
       if (!mbar_wait(&s.empty[stage], phase ^ 1u, w)) { ok = false; break; }
       const uint32_t bar = smem_addr(&s.full[stage]);
       mbar_arrive_expect_tx(&s.full[stage], kStageBytes);
-      load_operand(smem_addr(s.a + stage * kTileBytes), &maps.a[ti.prob], bar, q.a_mn, ti.m0,
-                   q.a_koff + kb * kBlockK);
-      load_operand(smem_addr(s.b + stage * kTileBytes), &maps.b[ti.prob], bar, q.b_mn, ti.n0,
-                   q.b_koff + kb * kBlockK);
+      load_operand(smem_addr(s.a + stage * kATileBytes), &maps.a[ti.prob], bar, q.a_mn, ti.m0,
+                   q.a_koff + kb * kBlockK, kBlockM);
+      load_operand(smem_addr(s.b + stage * kBTileBytes), &maps.b[ti.prob], bar, q.b_mn, ti.n0,
+                   q.b_koff + kb * kBlockK, kBlockN);
       pend_stage[n_issued % kStages] = stage;
       pend_par[n_issued % kStages] = phase;
       ++n_issued;
       if (++stage == kStages) { stage = 0; phase ^= 1u; }
     }
   }
-  if (!ok) {
-    const int n = min(n_issued, kStages);
-    for (int i = 0; i < n; ++i) {
-      const int j = (n_issued - 1 - i) % kStages;
-      const uint32_t a = smem_addr(&s.full[pend_stage[j]]);
-      const uint64_t t0 = global_timer_ns();
-      while (!mbar_test(a, pend_par[j]) && global_timer_ns() - t0 < 100000000ull) {
-      }
-    }
-  }
+  if (!ok) drain_loads(s, pend_stage, pend_par, n_issued);
 }
 
 __device__ __forceinline__ void gemm_mma(const GemmArgs& p, int nv, const SweepSmem& s, uint32_t tmem_base,
@@ -122,15 +112,15 @@ __device__ __forceinline__ void gemm_mma(const GemmArgs& p, int nv, const SweepS
   for (int tile = blockIdx.x; tile < nt && ok; tile += gridDim.x) {
     const TileInfo ti = tile_info(p, nv, tile);
     const GemmProb& q = p.prob[ti.prob];
-    const uint32_t idesc = make_idesc(128, 128, q.a_mn, q.b_mn);
+    const uint32_t idesc = make_idesc(kBlockM, kBlockN, q.a_mn, q.b_mn);
     if (!mbar_wait(&s.tempty[acc], acc_phase ^ 1u, w)) { ok = false; break; }
     tc_fence_after();
-    const uint32_t d = tmem_base + acc * 128;
+    const uint32_t d = tmem_base + acc * kBlockN;
     for (int kb = 0; kb < ti.nkb; ++kb) {
       if (!mbar_wait(&s.full[stage], phase, w)) { ok = false; break; }
       tc_fence_after();
-      const uint32_t sa = smem_addr(s.a + stage * kTileBytes);
-      const uint32_t sb = smem_addr(s.b + stage * kTileBytes);
+      const uint32_t sa = smem_addr(s.a + stage * kATileBytes);
+      const uint32_t sb = smem_addr(s.b + stage * kBTileBytes);
 #pragma unroll
       for (int j = 0; j < kBlockK / 16; ++j) {
         umma_bf16(d, operand_desc(sa, q.a_mn, j), operand_desc(sb, q.b_mn, j), idesc, (kb > 0 || j > 0) ? 1u : 0u);
@@ -143,19 +133,14 @@ __device__ __forceinline__ void gemm_mma(const GemmArgs& p, int nv, const SweepS
     acc ^= 1;
     if (acc == 0) acc_phase ^= 1u;
   }
-  if (!ok) {
-    umma_commit(smem_addr(s.drain));
-    const uint32_t a = smem_addr(s.drain);
-    const uint64_t t0 = global_timer_ns();
-    while (!mbar_test(a, 0) && global_timer_ns() - t0 < 100000000ull) {
-    }
-  }
+  if (!ok) drain_mma(s);
 }
 
 __device__ __forceinline__ void gemm_epilogue(const GemmArgs& p, int nv, const SweepSmem& s, uint32_t tmem_base,
                                               const WaitCtl& w) {
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int qq = warp & 3;
+  const int half = (warp - kEpiWarp0) >> 2;
   const uint32_t lane_addr = uint32_t(qq * 32) << 16;
   int acc = 0;
   uint32_t acc_phase = 0;
@@ -172,13 +157,13 @@ __device__ __forceinline__ void gemm_epilogue(const GemmArgs& p, int nv, const S
     }
     if (!mbar_wait(&s.tfull[acc], acc_phase, w)) return;
     tc_fence_after();
-    const uint32_t base = tmem_base + lane_addr + acc * 128;
+    const uint32_t base = tmem_base + lane_addr + acc * kBlockN + half * kHalfN;
 #pragma unroll 1
-    for (int ch = 0; ch < 4; ++ch) {
+    for (int ch = 0; ch < kHalfN / 32; ++ch) {
       float v[32];
       tmem_ld32(base + ch * 32, v);
       tmem_wait_ld();
-      if (ch == 3) {
+      if (ch == kHalfN / 32 - 1) {
         tc_fence_before();
         mbar_arrive(&s.tempty[acc]);
       }
@@ -186,7 +171,7 @@ __device__ __forceinline__ void gemm_epilogue(const GemmArgs& p, int nv, const S
 #pragma unroll
         for (int j = 0; j < 32; ++j) v[j] = 0.f;
       }
-      const int c0 = ti.n0 + ch * 32;
+      const int c0 = ti.n0 + half * kHalfN + ch * 32;
       if (!row_ok || c0 >= q.N) continue;
       float* dst = orow + c0;
       if (c0 + 32 <= q.N) {
@@ -213,18 +198,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
   extern __shared__ uint8_t smem_raw[];
   const SweepSmem s = carve_smem(smem_raw);
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  if (threadIdx.x == 0) {
-    for (int i = 0; i < kStages; ++i) {
-      mbar_init(&s.full[i], 1);
-      mbar_init(&s.empty[i], 1);
-    }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&s.tfull[i], 1);
-      mbar_init(&s.tempty[i], kEpiThreads);
-    }
-    mbar_init(s.drain, 1);
-    fence_mbar_init();
-  }
+  if (threadIdx.x == 0) init_barriers(s);
   if (warp == 0 && lane == 0) {
     for (int i = 0; i < p.nprob; ++i) {
       tma_prefetch_map(&maps.a[i]);
@@ -232,7 +206,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
     }
   }
   if (warp == 1) {
-    tmem_alloc(smem_addr(s.tmem_slot), 256);
+    tmem_alloc(smem_addr(s.tmem_slot), 2 * kBlockN);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -241,11 +215,12 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
   const uint32_t tmem_base = *s.tmem_slot;
   const int nv = *p.n_valid;
   const WaitCtl w{p.status, p.wait_limit_ns};
-  if (warp == 0) {
-    if (lane == 0) gemm_producer(maps, p, nv, s, w);
-  } else if (warp == 1) {
-    if (lane == 0) gemm_mma(p, nv, s, tmem_base, w);
+  if (warp < kEpiWarp0) {
+    regs_shrink<kRegsCtl>();
+    if (warp == 0 && lane == 0) gemm_producer(maps, p, nv, s, w);
+    if (warp == 1 && lane == 0) gemm_mma(p, nv, s, tmem_base, w);
   } else {
+    regs_grow<kRegsEpi>();
     gemm_epilogue(p, nv, s, tmem_base, w);
   }
   tc_fence_before();
@@ -253,7 +228,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
   if (warp == 1) {
     __syncwarp();
     tc_fence_after();
-    tmem_dealloc(tmem_base, 256);
+    tmem_dealloc(tmem_base, 2 * kBlockN);
   }
 }
 

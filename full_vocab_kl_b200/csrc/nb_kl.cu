@@ -27,7 +27,7 @@ using namespace nbkl;
 namespace {
 
 constexpr unsigned long long kWaitLimitNs = 1000000000ull;  // 1 s per pipeline wait
-constexpr int kTilesPerUnitFwd = 16;                         // 2048 vocabulary columns per split
+constexpr int kTilesPerUnitFwd = 8;                          // 2048 vocabulary columns per unit
 constexpr int64_t kDefaultChunkV = 8192;
 constexpr size_t kCtrlBytes = 256;
 
@@ -76,7 +76,7 @@ bool make_layout(const nb_kl_shape* sh, float beta, Layout& L) {
   if (sh->d_s % 8 || sh->d_t % 8) return false;
   if (sh->h_dtype != NB_BF16 && sh->h_dtype != NB_F32) return false;
   if (sh->reserved != 0) return false;
-  if (sh->chunk_v < 0 || (sh->chunk_v % 128) != 0) return false;
+  if (sh->chunk_v < 0 || (sh->chunk_v % kBlockN) != 0) return false;
   if (sh->n_tokens > (int64_t(1) << 30) || sh->vocab > (int64_t(1) << 30) || sh->d_s > 65536 || sh->d_t > 65536)
     return false;
   L.N = sh->n_tokens;
@@ -90,7 +90,7 @@ bool make_layout(const nb_kl_shape* sh, float beta, Layout& L) {
   L.lda_s = int64_t(L.kb_s) * kBlockK * (L.split ? 2 : 1);
   L.lda_t = int64_t(L.kb_t) * kBlockK * (L.split ? 2 : 1);
   L.n_vt = int((L.V + kBlockN - 1) / kBlockN);
-  L.n_split = (L.n_vt + kTilesPerUnitFwd - 1) / kTilesPerUnitFwd;
+  L.n_split = 2 * ((L.n_vt + kTilesPerUnitFwd - 1) / kTilesPerUnitFwd);  // two column halves per unit
   L.chunk_v = sh->chunk_v ? sh->chunk_v : std::min<int64_t>(kDefaultChunkV, round_up(L.V, kBlockN));
   const bool jsd = beta > 0.f && beta < 1.f;
   size_t off = kCtrlBytes;
@@ -159,6 +159,16 @@ nb_status device_info(DevInfo& out) {
       fail |= cudaFuncSetAttribute(sweep_kernel<kGradJsd>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes) != cudaSuccess;
       fail |= cudaFuncSetAttribute(gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes) != cudaSuccess;
       if (fail) return NB_ERR_CUDA;
+      // the warpgroup register split needs exactly the launch register count it was sized for
+      const void* fns[] = {(const void*)sweep_kernel<kStateNone>, (const void*)sweep_kernel<kStateS>,
+                           (const void*)sweep_kernel<kStateT>,    (const void*)sweep_kernel<kJsd>,
+                           (const void*)sweep_kernel<kGradFkl>,   (const void*)sweep_kernel<kGradRkl>,
+                           (const void*)sweep_kernel<kGradJsd>,   (const void*)gemm_kernel};
+      for (const void* f : fns) {
+        cudaFuncAttributes fa;
+        if (cudaFuncGetAttributes(&fa, f) != cudaSuccess) return NB_ERR_CUDA;
+        if (fa.numRegs < kRegsLaunch) d.ok = false;
+      }
     }
     d.attrs = true;
   }
@@ -249,7 +259,7 @@ void launch_gather(const Layout& L, const Ws& w, const void* h, int64_t d, __nv_
 bool sweep_maps(const Layout& L, const Ws& w, const void* W_s, const void* W_t, SweepMaps& m) {
   bool ok = true;
   ok &= make_map(&m.a_s, w.hs, L.lda_s, L.N_pad, L.lda_s * 2, kBlockK, kBlockM);
-  ok &= make_map(&m.b_s, W_s, L.d_s, L.V, L.d_s * 2, kBlockK, kBlockN);
+  ok &= make_map(&m.b_s, W_s, L.d_s, L.V, L.d_s * 2, kBlockK, kBlockN);  // 64 x 256 boxes
   ok &= make_map(&m.a_t, w.ht, L.lda_t, L.N_pad, L.lda_t * 2, kBlockK, kBlockM);
   ok &= make_map(&m.b_t, W_t, L.d_t, L.V, L.d_t * 2, kBlockK, kBlockN);
   return ok;
@@ -258,6 +268,7 @@ bool sweep_maps(const Layout& L, const Ws& w, const void* W_s, const void* W_t, 
 SweepArgs base_sweep_args(const Layout& L, const Ws& w, float beta, float tau) {
   SweepArgs a;
   std::memset(&a, 0, sizeof(a));
+  a.teacher_first = L.lda_t >= L.lda_s ? 1 : 0;
   a.V = int(L.V);
   a.v_begin = 0;
   a.v_end = int(L.V);
@@ -494,7 +505,7 @@ nb_status nb_kl_backward(const nb_kl_shape* shape, const void* h_s, const void* 
   dw.accumulate = accumulate_dW ? 1 : 0;
 
   const int n_tt_max = int(L.N_pad / kBlockM);
-  const int n_dt = int((L.d_s + kBlockN - 1) / kBlockN);
+  const int n_dt = int((L.d_s + kBlockN - 1) / kBlockN);   // 256-wide output column tiles
   for (int64_t v0 = 0; v0 < L.V; v0 += L.chunk_v) {
     const int64_t v1 = std::min(L.V, v0 + L.chunk_v);
     a.v_begin = int(v0);

@@ -3,17 +3,24 @@
 // "Nitrobrew tweet analysis", section "Nitrobrew 的两个动作": for each vocabulary
 // block, z_s = h_s W_s[v0:v1]^T and z_t = h_t W_t[v0:v1]^T are formed, the online
 // softmax / log-sum-exp accumulators and the KL terms are updated, and the block is
-// discarded. Here one block is a 128-token x 128-column tile: the student and the
-// teacher accumulators (128 TMEM columns each) live side by side in tensor memory,
-// double-buffered so that the epilogue of tile j overlaps the MMAs of tile j + 1.
+// discarded. Here one block is a 128-token x 256-column tile.
 //
-// Warp roles (192 threads, one CTA per SM, persistent over work units):
-//   warp 0  TMA producer: h and W tiles into a 6-stage shared-memory ring
-//   warp 1  MMA issuer: 4 x tcgen05.mma (K = 16) per 64-wide K block; owns TMEM
-//   warps 2-5  epilogue: tcgen05.ld of one token row per thread, base-2 online math
+// Tensor memory holds both fp32 accumulators of a tile (2 x 256 columns = all 512), so it
+// cannot be double-buffered. Instead the model with the larger K ("first") is multiplied
+// first; the epilogue copies the first accumulator into registers as soon as the tile is
+// complete and releases it, so the next tile's first-model MMAs run while the epilogue
+// streams the second accumulator. The second accumulator is released after its last read,
+// normally long before the next tile's first-model phase ends.
 //
-// A work unit is (token tile, run of `tiles_per_unit` vocabulary tiles); its per-token
-// partial state is written once per unit (the split-V partial LSE state).
+// Warp roles (384 threads, one CTA per SM, persistent over work units):
+//   warp 0     TMA producer: 128 x 64 h tiles and 256 x 64 W tiles into a 4-stage ring
+//   warp 1     MMA issuer: 4 x tcgen05.mma 128x256x16 per K block; owns TMEM
+//   warps 2-3  idle (warpgroup 0 hands its registers to the epilogue: 56 vs 224 per thread)
+//   warps 4-11 epilogue: two warps per TMEM lane quarter, each thread one token row and one
+//              128-column half of the tile, base-2 online math in registers
+//
+// A work unit is (token tile, run of `tiles_per_unit` vocabulary tiles); each thread writes
+// its row's partial state once per unit (split = 2 * unit + column half).
 #pragma once
 
 #include "common.cuh"
@@ -21,13 +28,13 @@
 namespace nbkl {
 
 struct SweepSmem {
-  uint8_t* a;          // kStages x 16 KB
-  uint8_t* b;          // kStages x 16 KB
-  uint64_t* full;      // kStages
-  uint64_t* empty;     // kStages
-  uint64_t* tfull;     // 2
-  uint64_t* tempty;    // 2
-  uint64_t* drain;     // 1
+  uint8_t* a;           // kStages x 16 KB
+  uint8_t* b;           // kStages x 32 KB
+  uint64_t* full;       // kStages
+  uint64_t* empty;      // kStages
+  uint64_t* tfull;      // tile complete (GEMM kernel: 2, one per accumulator stage)
+  uint64_t* tempty;     // accumulator released (sweep: [0] first model, [1] second model)
+  uint64_t* drain;      // 1
   uint32_t* tmem_slot;
 };
 
@@ -35,7 +42,7 @@ __device__ __forceinline__ SweepSmem carve_smem(uint8_t* raw) {
   SweepSmem s;
   uint8_t* base = align1024(raw);
   s.a = base;
-  s.b = base + kStages * kTileBytes;
+  s.b = base + kStages * kATileBytes;
   uint64_t* bars = reinterpret_cast<uint64_t*>(base + kStages * kStageBytes);
   s.full = bars;
   s.empty = bars + kStages;
@@ -44,6 +51,19 @@ __device__ __forceinline__ SweepSmem carve_smem(uint8_t* raw) {
   s.drain = bars + 2 * kStages + 4;
   s.tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * kStages + 5);
   return s;
+}
+
+__device__ __forceinline__ void init_barriers(const SweepSmem& s) {
+  for (int i = 0; i < kStages; ++i) {
+    mbar_init(&s.full[i], 1);
+    mbar_init(&s.empty[i], 1);
+  }
+  for (int i = 0; i < 2; ++i) {
+    mbar_init(&s.tfull[i], 1);
+    mbar_init(&s.tempty[i], kEpiThreads);
+  }
+  mbar_init(s.drain, 1);
+  fence_mbar_init();
 }
 
 struct UnitGrid {
@@ -60,31 +80,57 @@ __device__ __forceinline__ UnitGrid unit_grid(const SweepArgs& p) {
   return g;
 }
 
+// Bounded wait for the copies a failed producer may still have in flight.
+__device__ __forceinline__ void drain_loads(const SweepSmem& s, const uint32_t* pend_stage,
+                                            const uint32_t* pend_par, int n_issued) {
+  const int n = min(n_issued, kStages);
+  for (int i = 0; i < n; ++i) {
+    const int j = (n_issued - 1 - i) % kStages;
+    const uint32_t a = smem_addr(&s.full[pend_stage[j]]);
+    const uint64_t t0 = global_timer_ns();
+    while (!mbar_test(a, pend_par[j]) && global_timer_ns() - t0 < 100000000ull) {
+    }
+  }
+}
+
+// Bounded wait until every MMA this thread issued has completed.
+__device__ __forceinline__ void drain_mma(const SweepSmem& s) {
+  umma_commit(smem_addr(s.drain));
+  const uint32_t a = smem_addr(s.drain);
+  const uint64_t t0 = global_timer_ns();
+  while (!mbar_test(a, 0) && global_timer_ns() - t0 < 100000000ull) {
+  }
+}
+
 // ------------------------------------------------------------------ producer
 __device__ __forceinline__ void sweep_producer(const SweepMaps& maps, const SweepArgs& p, const UnitGrid& g,
                                                const SweepSmem& s, const WaitCtl& w) {
   int stage = 0;
   uint32_t phase = 0;
-  const int nkb = p.nkb_s + p.nkb_t;
-  uint32_t pend_stage[kStages];
-  uint32_t pend_par[kStages];
+  uint32_t pend_stage[kStages], pend_par[kStages];
   int n_issued = 0;
+  // first model = teacher when teacher_first
+  const CUtensorMap* a1 = p.teacher_first ? &maps.a_t : &maps.a_s;
+  const CUtensorMap* b1 = p.teacher_first ? &maps.b_t : &maps.b_s;
+  const CUtensorMap* a2 = p.teacher_first ? &maps.a_s : &maps.a_t;
+  const CUtensorMap* b2 = p.teacher_first ? &maps.b_s : &maps.b_t;
+  const int nk1 = p.teacher_first ? p.nkb_t : p.nkb_s, nk2 = p.teacher_first ? p.nkb_s : p.nkb_t;
+  const int bm1 = p.teacher_first ? p.bmod_t : p.bmod_s, bm2 = p.teacher_first ? p.bmod_s : p.bmod_t;
   bool ok = true;
   for (int u = blockIdx.x; u < g.n_units && ok; u += gridDim.x) {
     const int vu = u / g.n_tt, tt = u % g.n_tt;
     const int t_end = min((vu + 1) * p.tiles_per_unit, g.n_vt);
     for (int t = vu * p.tiles_per_unit; t < t_end && ok; ++t) {
       const int v0 = p.v_begin + t * kBlockN;
-      for (int kb = 0; kb < nkb; ++kb) {
+      for (int kb = 0; kb < nk1 + nk2; ++kb) {
         if (!mbar_wait(&s.empty[stage], phase ^ 1u, w)) { ok = false; break; }
-        const bool stu = kb < p.nkb_s;
-        const int k = stu ? kb : kb - p.nkb_s;
-        const int kbb = k % (stu ? p.bmod_s : p.bmod_t);
+        const bool one = kb < nk1;
+        const int k = one ? kb : kb - nk1;
+        const int kbb = k % (one ? bm1 : bm2);
         const uint32_t bar = smem_addr(&s.full[stage]);
         mbar_arrive_expect_tx(&s.full[stage], kStageBytes);
-        tma_load_2d(smem_addr(s.a + stage * kTileBytes), stu ? &maps.a_s : &maps.a_t, bar, k * kBlockK,
-                    tt * kBlockM);
-        tma_load_2d(smem_addr(s.b + stage * kTileBytes), stu ? &maps.b_s : &maps.b_t, bar, kbb * kBlockK, v0);
+        tma_load_2d(smem_addr(s.a + stage * kATileBytes), one ? a1 : a2, bar, k * kBlockK, tt * kBlockM);
+        tma_load_2d(smem_addr(s.b + stage * kBTileBytes), one ? b1 : b2, bar, kbb * kBlockK, v0);
         pend_stage[n_issued % kStages] = stage;
         pend_par[n_issued % kStages] = phase;
         ++n_issued;
@@ -92,17 +138,7 @@ __device__ __forceinline__ void sweep_producer(const SweepMaps& maps, const Swee
       }
     }
   }
-  if (!ok) {
-    // drain: wait (bounded) for the copies still in flight before the CTA can exit
-    const int n = min(n_issued, kStages);
-    for (int i = 0; i < n; ++i) {
-      const int j = (n_issued - 1 - i) % kStages;
-      const uint32_t a = smem_addr(&s.full[pend_stage[j]]);
-      const uint64_t t0 = global_timer_ns();
-      while (!mbar_test(a, pend_par[j]) && global_timer_ns() - t0 < 100000000ull) {
-      }
-    }
-  }
+  if (!ok) drain_loads(s, pend_stage, pend_par, n_issued);
 }
 
 // ------------------------------------------------------------------ MMA issuer
@@ -110,25 +146,26 @@ __device__ __forceinline__ void sweep_mma(const SweepArgs& p, const UnitGrid& g,
                                           uint32_t tmem_base, const WaitCtl& w) {
   int stage = 0;
   uint32_t phase = 0;
-  int acc = 0;
-  uint32_t acc_phase = 0;
-  const int nkb = p.nkb_s + p.nkb_t;
+  uint32_t lt = 0;  // tiles processed by this CTA
+  const int nk1 = p.teacher_first ? p.nkb_t : p.nkb_s, nk2 = p.teacher_first ? p.nkb_s : p.nkb_t;
   bool ok = true;
   for (int u = blockIdx.x; u < g.n_units && ok; u += gridDim.x) {
     const int vu = u / g.n_tt;
     const int t_end = min((vu + 1) * p.tiles_per_unit, g.n_vt);
-    for (int t = vu * p.tiles_per_unit; t < t_end && ok; ++t) {
-      if (!mbar_wait(&s.tempty[acc], acc_phase ^ 1u, w)) { ok = false; break; }
-      tc_fence_after();
-      const uint32_t d_s = tmem_base + acc * 256;
-      for (int kb = 0; kb < nkb; ++kb) {
+    for (int t = vu * p.tiles_per_unit; t < t_end && ok; ++t, ++lt) {
+      for (int kb = 0; kb < nk1 + nk2; ++kb) {
+        const bool one = kb < nk1;
+        const int k = one ? kb : kb - nk1;
+        if (k == 0) {
+          // the accumulator of this model must have been read by the epilogue
+          if (!mbar_wait(&s.tempty[one ? 0 : 1], (lt & 1u) ^ 1u, w)) { ok = false; break; }
+          tc_fence_after();
+        }
         if (!mbar_wait(&s.full[stage], phase, w)) { ok = false; break; }
         tc_fence_after();
-        const bool stu = kb < p.nkb_s;
-        const int k = stu ? kb : kb - p.nkb_s;
-        const uint32_t d = stu ? d_s : d_s + 128;
-        const uint32_t sa = smem_addr(s.a + stage * kTileBytes);
-        const uint32_t sb = smem_addr(s.b + stage * kTileBytes);
+        const uint32_t d = tmem_base + (one ? 0 : kBlockN);
+        const uint32_t sa = smem_addr(s.a + stage * kATileBytes);
+        const uint32_t sb = smem_addr(s.b + stage * kBTileBytes);
 #pragma unroll
         for (int j = 0; j < kBlockK / 16; ++j) {
           umma_bf16(d, make_sdesc(sa + j * 32, 16, 1024), make_sdesc(sb + j * 32, 16, 1024), kIdescKK,
@@ -138,19 +175,10 @@ __device__ __forceinline__ void sweep_mma(const SweepArgs& p, const UnitGrid& g,
         if (++stage == kStages) { stage = 0; phase ^= 1u; }
       }
       if (!ok) break;
-      umma_commit(smem_addr(&s.tfull[acc]));
-      acc ^= 1;
-      if (acc == 0) acc_phase ^= 1u;
+      umma_commit(smem_addr(&s.tfull[0]));
     }
   }
-  if (!ok) {
-    // make sure no MMA still writes TMEM before it is released
-    umma_commit(smem_addr(s.drain));
-    const uint32_t a = smem_addr(s.drain);
-    const uint64_t t0 = global_timer_ns();
-    while (!mbar_test(a, 0) && global_timer_ns() - t0 < 100000000ull) {
-    }
-  }
+  if (!ok) drain_mma(s);
 }
 
 // ------------------------------------------------------------------ epilogue math
@@ -257,16 +285,35 @@ __device__ __forceinline__ void chunk_grad(const float (&zs)[32], const float (&
     d4[q] = make_uint4(packed[4 * q], packed[4 * q + 1], packed[4 * q + 2], packed[4 * q + 3]);
 }
 
+template <int MODE>
+__device__ __forceinline__ void process_chunk(float (&zs)[32], float (&zt)[32], int n_ok, const SweepArgs& p,
+                                              const RowConst& c, float gs, RowState& r, float& js, float& ks,
+                                              __nv_bfloat16* gdst) {
+  const bool masked = n_ok < 32;
+  if (MODE <= kStateT) {
+    if (masked) chunk_state<MODE, true>(zs, zt, n_ok, p.scale, r);
+    else chunk_state<MODE, false>(zs, zt, n_ok, p.scale, r);
+  } else if (MODE == kJsd) {
+    if (masked) chunk_jsd<true>(zs, zt, n_ok, p.scale, c, js, ks);
+    else chunk_jsd<false>(zs, zt, n_ok, p.scale, c, js, ks);
+  } else {
+    if (masked) chunk_grad<MODE, true>(zs, zt, n_ok, p.scale, c, gs, gdst);
+    else chunk_grad<MODE, false>(zs, zt, n_ok, p.scale, c, gs, gdst);
+  }
+}
+
 // ------------------------------------------------------------------ epilogue
 template <int MODE>
 __device__ __forceinline__ void sweep_epilogue(const SweepArgs& p, const UnitGrid& g, const SweepSmem& s,
                                                uint32_t tmem_base, const WaitCtl& w) {
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int q = warp & 3;                      // TMEM lane quarter this warp may access
+  const int half = (warp - kEpiWarp0) >> 2;    // column half of the tile
   const int row_in_tile = q * 32 + lane;
   const uint32_t lane_addr = uint32_t(q * 32) << 16;
-  int acc = 0;
-  uint32_t acc_phase = 0;
+  const uint32_t col1 = tmem_base + lane_addr + half * kHalfN;   // first model
+  const uint32_t col2 = col1 + kBlockN;                          // second model
+  uint32_t lt = 0;
   RowConst c;
   c.beta = p.beta;
   c.omb = 1.0f - p.beta;
@@ -287,40 +334,33 @@ __device__ __forceinline__ void sweep_epilogue(const SweepArgs& p, const UnitGri
     RowState r{kNegBig, 0.f, kNegBig, 0.f, 0.f};
     float js = 0.f, ks = 0.f;
     const int t_end = min((vu + 1) * p.tiles_per_unit, g.n_vt);
-    for (int t = vu * p.tiles_per_unit; t < t_end; ++t) {
-      const int v0 = p.v_begin + t * kBlockN;
-      if (!mbar_wait(&s.tfull[acc], acc_phase, w)) return;
+    for (int t = vu * p.tiles_per_unit; t < t_end; ++t, ++lt) {
+      const int v0 = p.v_begin + t * kBlockN + half * kHalfN;
+      if (!mbar_wait(&s.tfull[0], lt & 1u, w)) return;
       tc_fence_after();
-      const uint32_t base = tmem_base + lane_addr + acc * 256;
-#pragma unroll 1
+      float F[4][32];
+#pragma unroll
+      for (int ch = 0; ch < 4; ++ch) tmem_ld32(col1 + ch * 32, F[ch]);
+      tmem_wait_ld();
+      tc_fence_before();
+      mbar_arrive(&s.tempty[0]);
+#pragma unroll
       for (int ch = 0; ch < 4; ++ch) {
-        float zs[32], zt[32];
-        tmem_ld32(base + ch * 32, zs);
-        tmem_ld32(base + 128 + ch * 32, zt);
+        float C[32];
+        tmem_ld32(col2 + ch * 32, C);
         tmem_wait_ld();
         if (ch == 3) {
           tc_fence_before();
-          mbar_arrive(&s.tempty[acc]);
+          mbar_arrive(&s.tempty[1]);
         }
         const int c0 = v0 + ch * 32;
-        const int n_ok = p.V - c0;          // columns of this chunk inside the vocabulary
-        const bool masked = n_ok < 32;
-        if (MODE <= kStateT) {
-          if (masked) chunk_state<MODE, true>(zs, zt, n_ok, p.scale, r);
-          else chunk_state<MODE, false>(zs, zt, n_ok, p.scale, r);
-        } else if (MODE == kJsd) {
-          if (masked) chunk_jsd<true>(zs, zt, n_ok, p.scale, c, js, ks);
-          else chunk_jsd<false>(zs, zt, n_ok, p.scale, c, js, ks);
-        } else {
-          __nv_bfloat16* dst = p.G + (long long)row * p.ldG + (c0 - p.v_begin);
-          if (masked) chunk_grad<MODE, true>(zs, zt, n_ok, p.scale, c, gs, dst);
-          else chunk_grad<MODE, false>(zs, zt, n_ok, p.scale, c, gs, dst);
-        }
+        const int n_ok = p.V - c0;            // columns of this chunk inside the vocabulary
+        __nv_bfloat16* gdst = (MODE >= kGradFkl) ? p.G + (long long)row * p.ldG + (c0 - p.v_begin) : nullptr;
+        if (p.teacher_first) process_chunk<MODE>(C, F[ch], n_ok, p, c, gs, r, js, ks, gdst);
+        else process_chunk<MODE>(F[ch], C, n_ok, p, c, gs, r, js, ks, gdst);
       }
-      acc ^= 1;
-      if (acc == 0) acc_phase ^= 1u;
     }
-    const long long off = (long long)vu * p.ld + row;
+    const long long off = (long long)(2 * vu + half) * p.ld + row;
     if (MODE <= kStateT) {
       p.out[off] = r.ms;
       p.out[p.field_stride + off] = r.ls;
@@ -340,18 +380,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   const SweepSmem s = carve_smem(smem_raw);
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  if (threadIdx.x == 0) {
-    for (int i = 0; i < kStages; ++i) {
-      mbar_init(&s.full[i], 1);
-      mbar_init(&s.empty[i], 1);
-    }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&s.tfull[i], 1);
-      mbar_init(&s.tempty[i], kEpiThreads);
-    }
-    mbar_init(s.drain, 1);
-    fence_mbar_init();
-  }
+  if (threadIdx.x == 0) init_barriers(s);
   if (warp == 0 && lane == 0) {
     tma_prefetch_map(&maps.a_s);
     tma_prefetch_map(&maps.b_s);
@@ -369,11 +398,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   const UnitGrid g = unit_grid(p);
   const WaitCtl w{p.status, p.wait_limit_ns};
 
-  if (warp == 0) {
-    if (lane == 0) sweep_producer(maps, p, g, s, w);
-  } else if (warp == 1) {
-    if (lane == 0) sweep_mma(p, g, s, tmem_base, w);
+  if (warp < kEpiWarp0) {
+    regs_shrink<kRegsCtl>();
+    if (warp == 0 && lane == 0) sweep_producer(maps, p, g, s, w);
+    if (warp == 1 && lane == 0) sweep_mma(p, g, s, tmem_base, w);
   } else {
+    regs_grow<kRegsEpi>();
     sweep_epilogue<MODE>(p, g, s, tmem_base, w);
   }
   tc_fence_before();
