@@ -73,9 +73,10 @@ def algorithmic_flops(w, n_valid):
 
 
 def kernel_source_sha():
+    """Hash of the device-code headers: a profile summary is only used while it matches."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "full_vocab_kl_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
+    for name in sorted(n for n in os.listdir(csrc) if n.endswith(".cuh")):
         with open(os.path.join(csrc, name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
