@@ -21,6 +21,7 @@ NB_ERR_CUDA = -4
 NB_ERR_TIMEOUT = -5
 NB_BF16 = 0
 NB_F32 = 1
+NOALLOC_SCRATCH_BYTES = 64 * 1024 * 1024
 
 # every function the header declares, with (restype, argtypes)
 SIGNATURES = {
@@ -31,6 +32,9 @@ SIGNATURES = {
     "nb_kl_backward": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_float, c_float,
                                c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_int, c_void_p,
                                c_size_t, c_void_p]),
+    "nb_kl_forward_noalloc": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_float,
+                                      c_float, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
+                                      c_void_p]),
     "nb_kl_status_string": (c_char_p, [c_int]),
     "nb_kl_device_status": (c_int, [c_void_p, c_void_p]),
     "nb_kl_debug_gemm": (c_int, [c_void_p, c_int, c_void_p, c_int, c_int64, c_int64, c_int64, c_void_p, c_void_p,

@@ -321,6 +321,28 @@ nb_status validate_common(const nb_kl_shape* shape, const void* h_s, const void*
   return NB_OK;
 }
 
+// ------------------------------------------------------------------ fixed scratch
+// Scratch of nb_kl_forward_noalloc: one array per device, created when the library's module
+// is loaded on that device and kept until the process exits. Its device address is looked up
+// once per device (with that device current) the first time the entry point runs there.
+static __device__ __align__(256) uint8_t g_fixed_scratch[NB_KL_NOALLOC_SCRATCH_BYTES];
+
+void* g_fixed_scratch_ptr[64] = {};
+std::mutex g_fixed_mu;
+
+nb_status fixed_scratch(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return NB_ERR_CUDA;
+  std::lock_guard<std::mutex> lk(g_fixed_mu);
+  if (!g_fixed_scratch_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_fixed_scratch) != cudaSuccess || p == nullptr) return NB_ERR_CUDA;
+    g_fixed_scratch_ptr[dev] = p;
+  }
+  *out = g_fixed_scratch_ptr[dev];
+  return NB_OK;
+}
+
 }  // namespace
 
 // =====================================================================================
@@ -523,6 +545,21 @@ nb_status nb_kl_backward(const nb_kl_shape* shape, const void* h_s, const void* 
     launch(gemm_kernel, dim3(std::max(1, std::min(dev.sms, tiles))), dim3(kThreads), size_t(kSmemBytes), st, gm, g);
   }
   return check_launch();
+}
+
+nb_status nb_kl_forward_noalloc(const nb_kl_shape* shape, const void* h_s, const void* W_s, const void* h_t,
+                                const void* W_t, const int64_t* labels, float beta, float tau, float* loss_tok,
+                                float* lse_s, float* lse_t, float* aux, float* loss_mean, int64_t* n_valid,
+                                void* stream) {
+  g_launches = 0;
+  const size_t need = nb_kl_workspace_size(shape, beta);
+  if (need == 0) return NB_ERR_INVALID_ARG;
+  if (need > size_t(NB_KL_NOALLOC_SCRATCH_BYTES)) return NB_ERR_WORKSPACE;
+  void* ws = nullptr;
+  const nb_status s = fixed_scratch(&ws);
+  if (s != NB_OK) return s;
+  return nb_kl_forward(shape, h_s, W_s, h_t, W_t, labels, beta, tau, loss_tok, lse_s, lse_t, aux, loss_mean,
+                       n_valid, ws, size_t(NB_KL_NOALLOC_SCRATCH_BYTES), stream);
 }
 
 nb_status nb_kl_debug_gemm(const void* A, int a_mn_major, const void* B, int b_mn_major, int64_t M, int64_t N,

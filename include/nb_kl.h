@@ -96,6 +96,28 @@ NB_KL_API nb_status nb_kl_backward(const nb_kl_shape* shape, const void* h_s, co
                          const float* lse_t, const float* aux, const float* grad_out, float* dh_s, float* dW_s,
                          int accumulate_dW, void* workspace, size_t workspace_bytes, void* stream);
 
+/* Size of the fixed device scratch behind nb_kl_forward_noalloc (64 MiB per device). */
+#define NB_KL_NOALLOC_SCRATCH_BYTES (64u * 1024u * 1024u)
+
+/* Forward without a caller-supplied workspace, for callers that cannot allocate device
+ * memory themselves: code that runs under a memory manager owning every device byte (a raw
+ * cudaMalloc would escape its accounting or fail its budget), or code that must not call
+ * cudaMalloc/cudaFree at all because those calls can synchronise the device. The pages have
+ * no counterpart; this is a deployment convenience.
+ * Same arguments and results as nb_kl_forward minus the workspace. The scratch is one fixed
+ * array of NB_KL_NOALLOC_SCRATCH_BYTES in the library's device image; every device that loads
+ * the library holds it until the process exits. Shapes whose nb_kl_workspace_size exceeds it
+ * return NB_ERR_WORKSPACE without launching anything. Nothing is allocated: the first call on
+ * a device looks up the array's device address (cudaGetSymbolAddress, with that device
+ * current) and caches it, so make that first call before any stream capture. All calls share
+ * the one array and it keeps the previous call's contents (the call clears what must start
+ * at zero): calls that may overlap on the GPU — from several streams or threads — race and
+ * must be serialised by the caller. */
+NB_KL_API nb_status nb_kl_forward_noalloc(const nb_kl_shape* shape, const void* h_s, const void* W_s,
+                                          const void* h_t, const void* W_t, const int64_t* labels, float beta,
+                                          float tau, float* loss_tok, float* lse_s, float* lse_t, float* aux,
+                                          float* loss_mean, int64_t* n_valid, void* stream);
+
 /* Static text for a status code. */
 NB_KL_API const char* nb_kl_status_string(nb_status status);
 
