@@ -262,7 +262,7 @@ def run_library(args):
 
     h_s, h_t, W_s, W_t = (to_dev(getattr(x, k)) for k in ("h_s", "h_t", "W_s", "W_t"))
     labels = torch.from_numpy(x.labels).to(dev)
-    shape = nb.make_shape(h_s, W_s, h_t, W_t, labels)
+    shape = nb.make_shape(h_s, W_s, h_t, W_t, labels, chunk_v=args.chunk_v)
     ws_bytes = nb.workspace_bytes(shape, w.beta)
     ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
     N = labels.shape[0]
@@ -276,10 +276,10 @@ def run_library(args):
     lib = _abi.lib()
 
     def step(hs, ht, lab):
-        nb.kl_forward(hs, W_s, ht, W_t, lab, w.beta, w.tau, workspace=ws, out=out)
+        nb.kl_forward(hs, W_s, ht, W_t, lab, w.beta, w.tau, workspace=ws, out=out, chunk_v=args.chunk_v)
         n1 = lib.nb_kl_last_launch_count()
         nb.kl_backward(hs, W_s, ht, W_t, lab, w.beta, w.tau, out["lse_s"], out["lse_t"], out["aux"], grad_out,
-                       dh_s=dh, dW_s=dW, accumulate_dW=w.accumulate_dW, workspace=ws)
+                       dh_s=dh, dW_s=dW, accumulate_dW=w.accumulate_dW, workspace=ws, chunk_v=args.chunk_v)
         return n1 + lib.nb_kl_last_launch_count()
 
     stream = torch.cuda.current_stream(dev)
@@ -382,7 +382,7 @@ def run_library(args):
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps},
             "gpu_launches": launches,
             "clocks": clk,
-            "scratch_bytes": ws_bytes, "peak_extra_alloc_bytes": int(peak_extra),
+            "scratch_bytes": ws_bytes, "peak_extra_alloc_bytes": int(peak_extra), "chunk_v": args.chunk_v,
         }
     if world > 1:
         dist.barrier()
@@ -402,6 +402,7 @@ def main():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD,
                     help="a workload name (synthetic.WORKLOADS) or a profiling-size one (synthetic.PROFILE_WORKLOADS)")
     ap.add_argument("--impl", default="library", choices=["library", "reference"])
+    ap.add_argument("--chunk-v", type=int, default=0, help="backward vocabulary chunk (0: library default)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:

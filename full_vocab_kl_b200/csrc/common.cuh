@@ -9,16 +9,22 @@
 
 namespace nbkl {
 
-// One CTA owns a 128-token x 256-column output tile (the MMA instruction is 128 x 256 x 16:
-// with N = 128 the tensor pipe stays busy for the same time and delivers half the work);
-// K advances 64 bf16 (one 128-byte swizzle row) per pipeline stage.
-constexpr int kBlockM = 128;
-constexpr int kBlockN = 256;
+// A pair of CTAs (a cluster of 2, one per SM) owns a 256-token x 256-column output tile: the
+// tcgen05 MMA is 256 x 256 x 16 with cta_group::2. Each CTA stages its own 128 rows of A and
+// 128 of the 256 rows of B (so an SM loads half of B per FLOP), and keeps its 128 rows of
+// the fp32 accumulators in its tensor memory. K advances 64 bf16 (one 128-byte swizzle row)
+// per pipeline stage. (A single-CTA 128 x 128 MMA keeps the tensor pipe as busy as a 128 x 256
+// one for half the work, and a single-CTA 128 x 256 GEMM reached only ~63% of cuBLAS here.)
+constexpr int kBlockM = 128;                           // rows per CTA
+constexpr int kPairM = 2 * kBlockM;                    // rows per pair (MMA M)
+constexpr int kBlockN = 256;                           // MMA N
+constexpr int kHalfB = kBlockN / 2;                    // B rows staged per CTA
 constexpr int kBlockK = 64;
-constexpr int kStages = 4;
+constexpr int kStages = 6;
 constexpr int kATileBytes = kBlockM * kBlockK * 2;     // 16 KB
-constexpr int kBTileBytes = kBlockN * kBlockK * 2;     // 32 KB
-constexpr int kStageBytes = kATileBytes + kBTileBytes; // 48 KB
+constexpr int kBTileBytes = kHalfB * kBlockK * 2;      // 16 KB
+constexpr int kStageBytes = kATileBytes + kBTileBytes; // 32 KB per CTA
+constexpr int kPairStageBytes = 2 * kStageBytes;       // bytes the leader's full barrier expects
 constexpr int kEpiWarps = 8;                           // two warps per TMEM lane quarter
 constexpr int kEpiWarp0 = 4;                           // epilogue = warpgroups 1 and 2
 constexpr int kEpiThreads = kEpiWarps * 32;
@@ -30,14 +36,20 @@ constexpr int kRegsCtl = 56;
 constexpr int kRegsEpi = 224;
 static_assert(128 * kRegsCtl + kEpiThreads * kRegsEpi <= kThreads * kRegsLaunch, "register split");
 constexpr int kHalfN = kBlockN / 2;                    // columns per epilogue thread per tile
-constexpr int kSmemBytes = kStages * kStageBytes + 1024 /*align*/ + 256 /*barriers*/;
+// Per epilogue warp, one 4 KB staging buffer for TMA stores (32 rows x 128 bytes, 128-byte
+// swizzle: fp32 32 x 32 chunks of the GEMM output, bf16 32 x 32 chunks of the gradient).
+constexpr int kStageOutBytes = 4096;
+constexpr int kSmemBytes = kStages * kStageBytes + kEpiWarps * kStageOutBytes + 1024 /*align*/ + 256 /*barriers*/;
+
+constexpr int kRing = 4;                               // work ids in flight inside a pair
+constexpr int kRingConsumers = 2 * (1 + 8);            // per CTA: MMA or TMA thread + 8 epilogue warps
 
 constexpr float kLn2 = 0.69314718055994530942f;
 constexpr float kLog2e = 1.44269504088896340736f;
 constexpr float kNegBig = -1.0e30f;  // finite "minus infinity" for masked columns
 
-// Idesc of the sweep's 128 x 256 K-major x K-major products.
-constexpr uint32_t kIdescKK = make_idesc(kBlockM, kBlockN, 0, 0);
+// Idesc of the sweep's 256 x 256 K-major x K-major pair products.
+constexpr uint32_t kIdescKK = make_idesc(kPairM, kBlockN, 0, 0);
 
 __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
   return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
@@ -56,6 +68,7 @@ enum SweepMode : int {
 
 struct SweepMaps {
   CUtensorMap a_s, b_s, a_t, b_t;   // compacted h_s, W_s, compacted h_t, W_t
+  CUtensorMap g_out;                // backward: gradient chunk, bf16, 32 x 32 boxes, 64-byte swizzle
 };
 
 struct SweepArgs {
@@ -78,6 +91,7 @@ struct SweepArgs {
   long long ldG;
   const float* gscale;    // device scalar grad_out / (N_v * tau)
   const int* n_valid;     // device scalar
+  int* sched;             // zeroed work counter: CTAs take units in order (null: static stride)
   int* status;
   unsigned long long wait_limit_ns;
 };
@@ -85,6 +99,7 @@ struct SweepArgs {
 // ------------------------------------------------------------------ backward GEMMs
 struct GemmMaps {
   CUtensorMap a[2], b[2];
+  CUtensorMap out[2];               // fp32 outputs, 32 x 32 boxes, 128-byte swizzle
 };
 
 struct GemmProb {
@@ -93,17 +108,15 @@ struct GemmProb {
   int m_dyn, M;            // m_dyn: M = n_valid (else M)
   int N;
   int k_dyn, K;            // k_dyn: K = round_up(n_valid, 128) (else K)
-  float* out;
-  long long ldo;
-  const int* row_map;      // output row of tile row m (null: row_off + m)
-  int row_off;
-  int accumulate;          // 1: out += acc, 0: out = acc
+  int out_row0;            // output-map row of tile row 0
+  int accumulate;          // 1: out += acc (TMA reduce-add), 0: out = acc (TMA store)
 };
 
 struct GemmArgs {
   GemmProb prob[2];
   int nprob;
   const int* n_valid;
+  int* sched;              // zeroed work counter (null: static stride)
   int* status;
   unsigned long long wait_limit_ns;
 };

@@ -16,7 +16,7 @@
 #include <mutex>
 #include <vector>
 
-#include "../../include/nb_kl.h"
+#include "nb_kl.h"
 #include "common.cuh"
 #include "gemm.cuh"
 #include "rowops.cuh"
@@ -28,7 +28,6 @@ namespace {
 
 constexpr unsigned long long kWaitLimitNs = 1000000000ull;  // 1 s per pipeline wait
 constexpr int kTilesPerUnitFwd = 8;                          // 2048 vocabulary columns per unit
-constexpr int64_t kDefaultChunkV = 8192;
 constexpr size_t kCtrlBytes = 256;
 
 thread_local int g_launches = 0;
@@ -66,7 +65,9 @@ struct Layout {
   int64_t lda_s, lda_t;  // row length of the compacted h buffers
   int n_vt, n_split;
   int64_t chunk_v;
-  size_t off_idx, off_hs, off_ht, off_rl2s, off_rl2t, off_raux, off_state, off_part, off_G, total;
+  int n_chunks;          // backward vocabulary chunks
+  size_t off_idx, off_hs, off_ht, off_rl2s, off_rl2t, off_raux, off_sched, off_dhc, off_state, off_part, off_G,
+      g_bytes, total;
   long long fs_state;    // elements between state fields
 };
 
@@ -80,7 +81,7 @@ bool make_layout(const nb_kl_shape* sh, float beta, Layout& L) {
   if (sh->n_tokens > (int64_t(1) << 30) || sh->vocab > (int64_t(1) << 30) || sh->d_s > 65536 || sh->d_t > 65536)
     return false;
   L.N = sh->n_tokens;
-  L.N_pad = round_up(std::max<int64_t>(L.N, 1), kBlockM);
+  L.N_pad = round_up(std::max<int64_t>(L.N, 1), kPairM);
   L.V = sh->vocab;
   L.d_s = sh->d_s;
   L.d_t = sh->d_t;
@@ -91,7 +92,12 @@ bool make_layout(const nb_kl_shape* sh, float beta, Layout& L) {
   L.lda_t = int64_t(L.kb_t) * kBlockK * (L.split ? 2 : 1);
   L.n_vt = int((L.V + kBlockN - 1) / kBlockN);
   L.n_split = 2 * ((L.n_vt + kTilesPerUnitFwd - 1) / kTilesPerUnitFwd);  // two column halves per unit
-  L.chunk_v = sh->chunk_v ? sh->chunk_v : std::min<int64_t>(kDefaultChunkV, round_up(L.V, kBlockN));
+  // default chunk: about 4096 gradient tiles per sweep launch (so the two gradient buffers
+  // take ~0.5 GB whatever the token count), between 2048 and 32768 columns
+  const int64_t auto_chunk = round_up(std::max<int64_t>(2048, std::min<int64_t>(32768, (int64_t(1) << 20) /
+                                                                                    (L.N_pad / kBlockM))),
+                                      kBlockN);  // 128-row halves of the pair tiles
+  L.chunk_v = sh->chunk_v ? sh->chunk_v : std::min<int64_t>(auto_chunk, round_up(L.V, kBlockN));
   const bool jsd = beta > 0.f && beta < 1.f;
   size_t off = kCtrlBytes;
   L.off_idx = off;   off = align256(off + size_t(L.N_pad) * 4);
@@ -100,14 +106,17 @@ bool make_layout(const nb_kl_shape* sh, float beta, Layout& L) {
   L.off_rl2s = off;  off = align256(off + size_t(L.N_pad) * 4);
   L.off_rl2t = off;  off = align256(off + size_t(L.N_pad) * 4);
   L.off_raux = off;  off = align256(off + size_t(L.N_pad) * 4);
-  // the forward's split state and the backward's gradient chunk share one region
+  L.n_chunks = int((L.V + L.chunk_v - 1) / L.chunk_v);
+  L.off_sched = off; off = align256(off + size_t(2 * L.n_chunks + 2) * 4);   // one work counter per launch
+  L.off_dhc = off;   off = align256(off + size_t(L.N_pad) * L.d_s * 4);        // compacted dh_s (backward)
+  // the forward's split state and the backward's two gradient-chunk buffers share one region
   const size_t state_bytes = align256(size_t(5) * L.n_split * L.N_pad * 4);
   const size_t part_bytes = jsd ? align256(size_t(2) * L.n_split * L.N_pad * 4) : 0;
-  const size_t g_bytes = align256(size_t(L.N_pad) * L.chunk_v * 2);
+  L.g_bytes = align256(size_t(L.N_pad) * L.chunk_v * 2);
   L.off_state = off;
   L.off_part = off + state_bytes;
   L.off_G = off;
-  off += std::max(state_bytes + part_bytes, g_bytes);
+  off += std::max(state_bytes + part_bytes, 2 * L.g_bytes);
   L.total = off;
   L.fs_state = (long long)L.n_split * L.N_pad;
   return true;
@@ -131,9 +140,32 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 
 struct DevInfo {
   int sms = 0;
+  int pairs = 0;         // CTA pairs (clusters of 2) that can be resident at once
   bool ok = false;
   bool attrs = false;
 };
+
+// Second stream of the backward (the GEMMs of chunk c overlap the gradient sweep of chunk
+// c + 1) and its events: one set per host thread and device, created on first use.
+struct AuxStream {
+  cudaStream_t aux = nullptr;
+  cudaEvent_t fork = nullptr, join = nullptr, swept[2] = {nullptr, nullptr}, used[2] = {nullptr, nullptr};
+};
+thread_local AuxStream g_aux[64];
+
+nb_status aux_stream(AuxStream** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return NB_ERR_CUDA;
+  AuxStream& a = g_aux[dev];
+  if (!a.aux) {
+    if (cudaStreamCreateWithFlags(&a.aux, cudaStreamNonBlocking) != cudaSuccess) return NB_ERR_CUDA;
+    cudaEvent_t* evs[] = {&a.fork, &a.join, &a.swept[0], &a.swept[1], &a.used[0], &a.used[1]};
+    for (cudaEvent_t* e : evs)
+      if (cudaEventCreateWithFlags(e, cudaEventDisableTiming) != cudaSuccess) return NB_ERR_CUDA;
+  }
+  *out = &a;
+  return NB_OK;
+}
 DevInfo g_dev[64];
 std::mutex g_dev_mu;
 
@@ -169,6 +201,23 @@ nb_status device_info(DevInfo& out) {
         if (cudaFuncGetAttributes(&fa, f) != cudaSuccess) return NB_ERR_CUDA;
         if (fa.numRegs < kRegsLaunch) d.ok = false;
       }
+      // persistent grids: as many pairs as fit at once (a cluster stays inside one GPC)
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3(2 * (sms / 2));
+      cfg.blockDim = dim3(kThreads);
+      cfg.dynamicSmemBytes = kSmemBytes;
+      cudaLaunchAttribute attr;
+      attr.id = cudaLaunchAttributeClusterDimension;
+      attr.val.clusterDim.x = 2;
+      attr.val.clusterDim.y = 1;
+      attr.val.clusterDim.z = 1;
+      cfg.attrs = &attr;
+      cfg.numAttrs = 1;
+      int clusters = 0;
+      if (cudaOccupancyMaxActiveClusters(&clusters, (const void*)sweep_kernel<kStateS>, &cfg) != cudaSuccess ||
+          clusters < 1)
+        clusters = sms / 2;
+      d.pairs = std::min(clusters, sms / 2);
     }
     d.attrs = true;
   }
@@ -176,18 +225,25 @@ nb_status device_info(DevInfo& out) {
   return d.ok ? NB_OK : NB_ERR_UNSUPPORTED;
 }
 
-// 2-D bf16 tensor map with 128-byte swizzle; out-of-range elements read as zero.
+// 2-D tensor map; loads read out-of-range elements as zero, stores skip them.
 bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint64_t row_bytes,
-              uint32_t box_inner, uint32_t box_outer) {
+              uint32_t box_inner, uint32_t box_outer,
+              CUtensorMapDataType dtype = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
+              CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_128B) {
   auto enc = encode_fn();
   if (!enc) return false;
   cuuint64_t dims[2] = {inner, outer};
   cuuint64_t strides[1] = {row_bytes};
   cuuint32_t box[2] = {box_inner, box_outer};
   cuuint32_t es[2] = {1, 1};
-  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
-             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  return enc(m, dtype, 2, const_cast<void*>(base), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// fp32 output map with 32 x 32 boxes (128-byte rows, 128-byte swizzle) for the GEMM epilogue
+bool make_out_map(CUtensorMap* m, float* base, uint64_t cols, uint64_t rows) {
+  return make_map(m, base, cols, rows, cols * 4, 32, 32, CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
+                  CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
@@ -217,6 +273,8 @@ nb_status check_launch() { return cudaGetLastError() == cudaSuccess ? NB_OK : NB
 struct Ws {
   Ctrl* ctrl;
   int* idx;
+  int* sched;
+  float* dhc;
   __nv_bfloat16 *hs, *ht;
   float *rl2s, *rl2t, *raux, *state, *part;
   __nv_bfloat16* G;
@@ -227,6 +285,8 @@ Ws carve(const Layout& L, void* ws) {
   Ws w;
   w.ctrl = reinterpret_cast<Ctrl*>(b);
   w.idx = reinterpret_cast<int*>(b + L.off_idx);
+  w.sched = reinterpret_cast<int*>(b + L.off_sched);
+  w.dhc = reinterpret_cast<float*>(b + L.off_dhc);
   w.hs = reinterpret_cast<__nv_bfloat16*>(b + L.off_hs);
   w.ht = reinterpret_cast<__nv_bfloat16*>(b + L.off_ht);
   w.rl2s = reinterpret_cast<float*>(b + L.off_rl2s);
@@ -259,9 +319,9 @@ void launch_gather(const Layout& L, const Ws& w, const void* h, int64_t d, __nv_
 bool sweep_maps(const Layout& L, const Ws& w, const void* W_s, const void* W_t, SweepMaps& m) {
   bool ok = true;
   ok &= make_map(&m.a_s, w.hs, L.lda_s, L.N_pad, L.lda_s * 2, kBlockK, kBlockM);
-  ok &= make_map(&m.b_s, W_s, L.d_s, L.V, L.d_s * 2, kBlockK, kBlockN);  // 64 x 256 boxes
+  ok &= make_map(&m.b_s, W_s, L.d_s, L.V, L.d_s * 2, kBlockK, kHalfB);  // each CTA: 128 W rows
   ok &= make_map(&m.a_t, w.ht, L.lda_t, L.N_pad, L.lda_t * 2, kBlockK, kBlockM);
-  ok &= make_map(&m.b_t, W_t, L.d_t, L.V, L.d_t * 2, kBlockK, kBlockN);
+  ok &= make_map(&m.b_t, W_t, L.d_t, L.V, L.d_t * 2, kBlockK, kHalfB);
   return ok;
 }
 
@@ -293,17 +353,23 @@ SweepArgs base_sweep_args(const Layout& L, const Ws& w, float beta, float tau) {
   return a;
 }
 
-int sweep_grid(const DevInfo& dev, const Layout& L, const SweepArgs& a) {
-  const int n_tt = int(L.N_pad / kBlockM);
+// grid of a pair kernel: 2 CTAs per pair, at most one resident wave of pairs
+unsigned pair_grid(const DevInfo& dev, int work_items) {
+  return unsigned(2 * std::max(1, std::min(dev.pairs, work_items)));
+}
+
+int sweep_units(const Layout& L, const SweepArgs& a) {
+  const int n_tt = int(L.N_pad / kPairM);
   const int n_vt = (a.v_end - a.v_begin + kBlockN - 1) / kBlockN;
   const int n_vu = (n_vt + a.tiles_per_unit - 1) / a.tiles_per_unit;
-  return std::max(1, std::min(dev.sms, n_tt * n_vu));
+  return n_tt * n_vu;
 }
 
 template <int MODE>
 void launch_sweep(const DevInfo& dev, const Layout& L, const SweepMaps& m, const SweepArgs& a, cudaStream_t st) {
   next_cat(MODE <= kStateT ? NB_KL_KERNEL_SWEEP_FWD : MODE == kJsd ? NB_KL_KERNEL_SWEEP_JSD : NB_KL_KERNEL_SWEEP_GRAD);
-  launch(sweep_kernel<MODE>, dim3(sweep_grid(dev, L, a)), dim3(kThreads), size_t(kSmemBytes), st, m, a);
+  launch(sweep_kernel<MODE>, dim3(pair_grid(dev, sweep_units(L, a))), dim3(kThreads), size_t(kSmemBytes), st, m,
+         a);
 }
 
 nb_status validate_common(const nb_kl_shape* shape, const void* h_s, const void* W_s, const void* h_t,
@@ -432,10 +498,12 @@ nb_status nb_kl_forward(const nb_kl_shape* shape, const void* h_s, const void* W
   launch_gather(L, w, h_s, L.d_s, w.hs, L.lda_s, st);
   launch_gather(L, w, h_t, L.d_t, w.ht, L.lda_t, st);
 
+  if (cudaMemsetAsync(w.sched, 0, size_t(2 * L.n_chunks + 2) * 4, st) != cudaSuccess) return NB_ERR_CUDA;
   SweepMaps maps;
   if (!sweep_maps(L, w, W_s, W_t, maps)) return NB_ERR_CUDA;
   SweepArgs a = base_sweep_args(L, w, beta, tau);
   a.out = w.state;
+  a.sched = w.sched;
   int kl_dir = 0;
   if (beta == 1.f) {
     launch_sweep<kStateS>(dev, L, maps, a, st);
@@ -446,14 +514,15 @@ nb_status nb_kl_forward(const nb_kl_shape* shape, const void* h_s, const void* W
   } else {
     launch_sweep<kStateNone>(dev, L, maps, a, st);
   }
-  const unsigned rb = unsigned((L.N_pad + 255) / 256);
-  launch(merge_kernel, dim3(rb), dim3(256), 0, st, (const float*)w.state, (long long)L.fs_state, int(L.N_pad),
+  const unsigned rb = unsigned((L.N_pad + kMergeRows - 1) / kMergeRows);
+  launch(merge_kernel, dim3(rb), dim3(kMergeRows * kMergeLanes), 0, st, (const float*)w.state, (long long)L.fs_state, int(L.N_pad),
          L.n_split, (const int*)w.idx, (const Ctrl*)w.ctrl, kl_dir, loss_tok, lse_s, lse_t, aux, w.rl2s, w.rl2t);
   if (kl_dir == 0) {
     SweepArgs b = a;
     b.out = w.part;
+    b.sched = w.sched + 1;
     launch_sweep<kJsd>(dev, L, maps, b, st);
-    launch(jsd_finalize_kernel, dim3(rb), dim3(256), 0, st, (const float*)w.part, (long long)L.fs_state,
+    launch(jsd_finalize_kernel, dim3(rb), dim3(kMergeRows * kMergeLanes), 0, st, (const float*)w.part, (long long)L.fs_state,
            int(L.N_pad), L.n_split, (const int*)w.idx, (const Ctrl*)w.ctrl, loss_tok, aux);
   }
   launch(mean_kernel, dim3(1), dim3(1024), 0, st, (const float*)loss_tok, int(L.N), (const Ctrl*)w.ctrl,
@@ -488,20 +557,29 @@ nb_status nb_kl_backward(const nb_kl_shape* shape, const void* h_s, const void* 
   launch(zero_masked_rows_kernel, dim3(unsigned(L.N)), dim3(128), 0, st, labels, (long long)shape->ignore_index,
          dh_s, int(L.d_s));
 
-  SweepMaps maps;
-  if (!sweep_maps(L, w, W_s, W_t, maps)) return NB_ERR_CUDA;
-  GemmMaps gm;
+  if (cudaMemsetAsync(w.sched, 0, size_t(2 * L.n_chunks + 2) * 4, st) != cudaSuccess) return NB_ERR_CUDA;
+  // two gradient-chunk buffers: the sweep of chunk c + 1 may run while the GEMMs of chunk c read
+  __nv_bfloat16* gbuf[2] = {w.G, reinterpret_cast<__nv_bfloat16*>(reinterpret_cast<uint8_t*>(w.G) + L.g_bytes)};
+  SweepMaps maps[2];
+  GemmMaps gm[2];
   bool ok = true;
-  // dh_s: A = G (K-major, box 64 x 128), B = W_s chunk as K x N (MN-major, 64 x 64 boxes)
-  ok &= make_map(&gm.a[0], w.G, L.chunk_v, L.N_pad, L.chunk_v * 2, kBlockK, kBlockM);
-  ok &= make_map(&gm.b[0], W_s, L.d_s, L.V, L.d_s * 2, 64, 64);
-  // dW_s: A = G^T (MN-major), B = compacted h_s (hi part) as K x N (MN-major)
-  ok &= make_map(&gm.a[1], w.G, L.chunk_v, L.N_pad, L.chunk_v * 2, 64, 64);
-  ok &= make_map(&gm.b[1], w.hs, L.d_s, L.N_pad, L.lda_s * 2, 64, 64);
+  for (int b = 0; b < 2; ++b) {
+    ok &= sweep_maps(L, w, W_s, W_t, maps[b]);
+    // gradient chunk written by the sweep epilogue: bf16 32 x 32 boxes, 64-byte rows
+    ok &= make_map(&maps[b].g_out, gbuf[b], L.chunk_v, L.N_pad, L.chunk_v * 2, 32, 32,
+                   CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, CU_TENSOR_MAP_SWIZZLE_64B);
+    ok &= make_out_map(&gm[b].out[0], w.dhc, L.d_s, L.N_pad);
+    ok &= make_out_map(&gm[b].out[1], dW_s, L.d_s, L.V);
+    // dh_s: A = G (K-major, box 64 x 128), B = W_s chunk as K x N (MN-major, 64 x 64 boxes)
+    ok &= make_map(&gm[b].a[0], gbuf[b], L.chunk_v, L.N_pad, L.chunk_v * 2, kBlockK, kBlockM);
+    ok &= make_map(&gm[b].b[0], W_s, L.d_s, L.V, L.d_s * 2, 64, 64);
+    // dW_s: A = G^T (MN-major), B = compacted h_s (hi part) as K x N (MN-major)
+    ok &= make_map(&gm[b].a[1], gbuf[b], L.chunk_v, L.N_pad, L.chunk_v * 2, 64, 64);
+    ok &= make_map(&gm[b].b[1], w.hs, L.d_s, L.N_pad, L.lda_s * 2, 64, 64);
+  }
   if (!ok) return NB_ERR_CUDA;
 
   SweepArgs a = base_sweep_args(L, w, beta, tau);
-  a.G = w.G;
   a.ldG = L.chunk_v;
   a.tiles_per_unit = 1;
   GemmArgs g;
@@ -515,35 +593,56 @@ nb_status nb_kl_backward(const nb_kl_shape* shape, const void* h_s, const void* 
   dh.b_mn = 1;
   dh.m_dyn = 1;
   dh.N = int(L.d_s);
-  dh.out = dh_s;
-  dh.ldo = L.d_s;
-  dh.row_map = w.idx;
+  dh.out_row0 = 0;
   GemmProb& dw = g.prob[1];
   dw.a_mn = 1;
   dw.b_mn = 1;
   dw.N = int(L.d_s);
   dw.k_dyn = 1;
-  dw.ldo = L.d_s;
   dw.accumulate = accumulate_dW ? 1 : 0;
 
-  const int n_tt_max = int(L.N_pad / kBlockM);
+  const int n_tt_max = int(L.N_pad / kPairM);
   const int n_dt = int((L.d_s + kBlockN - 1) / kBlockN);   // 256-wide output column tiles
-  for (int64_t v0 = 0; v0 < L.V; v0 += L.chunk_v) {
-    const int64_t v1 = std::min(L.V, v0 + L.chunk_v);
+  AuxStream* ax = nullptr;
+  if ((s = aux_stream(&ax)) != NB_OK) return s;
+  // fork: the GEMMs run on a second stream, ordered after everything before this call
+  if (cudaEventRecord(ax->fork, st) != cudaSuccess || cudaStreamWaitEvent(ax->aux, ax->fork, 0) != cudaSuccess)
+    return NB_ERR_CUDA;
+  bool enq = true;
+  for (int c = 0; c < L.n_chunks && enq; ++c) {
+    const int b = c & 1;
+    const int64_t v0 = int64_t(c) * L.chunk_v, v1 = std::min(L.V, v0 + L.chunk_v);
+    // buffer b was last read by the GEMMs of chunk c - 2
+    if (c >= 2 && cudaStreamWaitEvent(st, ax->used[b], 0) != cudaSuccess) { enq = false; break; }
     a.v_begin = int(v0);
     a.v_end = int(v1);
-    if (beta == 0.f) launch_sweep<kGradFkl>(dev, L, maps, a, st);
-    else if (beta == 1.f) launch_sweep<kGradRkl>(dev, L, maps, a, st);
-    else launch_sweep<kGradJsd>(dev, L, maps, a, st);
+    a.G = gbuf[b];
+    a.sched = w.sched + 2 * c;
+    if (beta == 0.f) launch_sweep<kGradFkl>(dev, L, maps[b], a, st);
+    else if (beta == 1.f) launch_sweep<kGradRkl>(dev, L, maps[b], a, st);
+    else launch_sweep<kGradJsd>(dev, L, maps[b], a, st);
+    if (cudaEventRecord(ax->swept[b], st) != cudaSuccess ||
+        cudaStreamWaitEvent(ax->aux, ax->swept[b], 0) != cudaSuccess) {
+      enq = false;
+      break;
+    }
     dh.K = int(v1 - v0);
     dh.b_koff = int(v0);
-    dh.accumulate = v0 > 0 ? 1 : 0;
+    dh.accumulate = c > 0 ? 1 : 0;
     dw.M = int(v1 - v0);
-    dw.out = dW_s + v0 * L.d_s;
-    const int tiles = n_tt_max * n_dt + int((v1 - v0 + kBlockM - 1) / kBlockM) * n_dt;
+    dw.out_row0 = int(v0);
+    g.sched = w.sched + 2 * c + 1;
+    const int tiles = n_tt_max * n_dt + int((v1 - v0 + kPairM - 1) / kPairM) * n_dt;
     next_cat(NB_KL_KERNEL_GEMM_BWD);
-    launch(gemm_kernel, dim3(std::max(1, std::min(dev.sms, tiles))), dim3(kThreads), size_t(kSmemBytes), st, gm, g);
+    launch(gemm_kernel, dim3(pair_grid(dev, tiles)), dim3(kThreads), size_t(kSmemBytes), ax->aux, gm[b], g);
+    if (cudaEventRecord(ax->used[b], ax->aux) != cudaSuccess) enq = false;
   }
+  if (enq) launch(scatter_rows_kernel, dim3(unsigned(L.N_pad)), dim3(128), 0, ax->aux, (const float*)w.dhc,
+                  int(L.d_s), dh_s, (const int*)w.idx, (const Ctrl*)w.ctrl);
+  // join (also after a failure part-way): work after this call on `st` sees every GEMM result
+  if (cudaEventRecord(ax->join, ax->aux) != cudaSuccess || cudaStreamWaitEvent(st, ax->join, 0) != cudaSuccess)
+    return NB_ERR_CUDA;
+  if (!enq) return NB_ERR_CUDA;
   return check_launch();
 }
 
@@ -580,7 +679,7 @@ nb_status nb_kl_debug_gemm(const void* A, int a_mn_major, const void* B, int b_m
   bool ok = true;
   if (!a_mn_major) ok &= make_map(&gm.a[0], A, K, M, K * 2, kBlockK, kBlockM);
   else ok &= make_map(&gm.a[0], A, M, K, M * 2, 64, 64);
-  if (!b_mn_major) ok &= make_map(&gm.b[0], B, K, N, K * 2, kBlockK, kBlockN);
+  if (!b_mn_major) ok &= make_map(&gm.b[0], B, K, N, K * 2, kBlockK, kHalfB);
   else ok &= make_map(&gm.b[0], B, N, K, N * 2, 64, 64);
   if (!ok) return NB_ERR_CUDA;
   GemmArgs g;
@@ -595,10 +694,10 @@ nb_status nb_kl_debug_gemm(const void* A, int a_mn_major, const void* B, int b_m
   q.M = int(M);
   q.N = int(N);
   q.K = int(K);
-  q.out = C;
-  q.ldo = N;
-  const int tiles = int((M + kBlockM - 1) / kBlockM * ((N + kBlockN - 1) / kBlockN));
-  launch(gemm_kernel, dim3(std::max(1, std::min(dev.sms, tiles))), dim3(kThreads), size_t(kSmemBytes), st, gm, g);
+  ok = make_out_map(&gm.out[0], C, N, M);
+  if (!ok) return NB_ERR_CUDA;
+  const int tiles = int((M + kPairM - 1) / kPairM * ((N + kBlockN - 1) / kBlockN));
+  launch(gemm_kernel, dim3(pair_grid(dev, tiles)), dim3(kThreads), size_t(kSmemBytes), st, gm, g);
   return check_launch();
 }
 

@@ -65,7 +65,7 @@ __global__ void __launch_bounds__(kScanThreads) compact_kernel(const int64_t* __
 
 // ------------------------------------------------------------------ gather of valid rows
 // dst row i (< n_valid) = src row idx[i] as bf16, zero-padded to `lda` columns; rows
-// n_valid .. round_up(n_valid, 128) are zeroed. With `split`, an fp32 source is stored as
+// n_valid .. round_up(n_valid, 256) (the last pair tile) are zeroed. With `split`, an fp32 source is stored as
 // [hi | lo] with hi = bf16(x) and lo = bf16(x - hi), each half `half` columns wide, so that
 // hi*W + lo*W carries x to about 16 bits.
 template <bool F32_SRC>
@@ -76,7 +76,7 @@ __global__ void gather_rows_kernel(const void* __restrict__ src, int d, __nv_bfl
                                    float* row_l2t, float* row_aux) {
   const int i = blockIdx.x;
   const int nv = ctrl->n_valid;
-  const int rows_needed = ((nv + kBlockM - 1) / kBlockM) * kBlockM;
+  const int rows_needed = ((nv + kPairM - 1) / kPairM) * kPairM;
   if (i >= rows_needed) return;
   __nv_bfloat16* out = dst + (long long)i * lda;
   const bool live = i < nv;
@@ -112,59 +112,103 @@ __global__ void gather_rows_kernel(const void* __restrict__ src, int d, __nv_bfl
 //   LSE(u) = ln 2 * (m + log2 l),  KL = ln 2 * (a / l_p - L2_p + L2_q)
 // `kl_dir`: 1 reverse (p = student), 2 forward (p = teacher), 0 none (JSD pass 1: the
 // base-2 LSEs go to row_l2s / row_l2t for the second pass).
-__global__ void merge_kernel(const float* __restrict__ state, long long fs, int ld, int n_split,
-                             const int* __restrict__ idx, const Ctrl* __restrict__ ctrl, int kl_dir,
-                             float* loss_tok, float* lse_s, float* lse_t, float* aux, float* row_l2s,
-                             float* row_l2t) {
-  const int i = blockIdx.x * blockDim.x + threadIdx.x;
-  if (i >= ctrl->n_valid) return;
+// Block = 32 rows x 8 split lanes: lane j of row r visits splits j, j + 8, ... so that a warp
+// (32 consecutive rows, one split) reads contiguous memory; the 8 partial results of a row
+// are combined in shared memory in a fixed order.
+constexpr int kMergeRows = 32, kMergeLanes = 8;
+
+__global__ void __launch_bounds__(kMergeRows * kMergeLanes)
+    merge_kernel(const float* __restrict__ state, long long fs, int ld, int n_split, const int* __restrict__ idx,
+                 const Ctrl* __restrict__ ctrl, int kl_dir, float* loss_tok, float* lse_s, float* lse_t, float* aux,
+                 float* row_l2s, float* row_l2t) {
+  __shared__ float sm_s[kMergeLanes][kMergeRows], sm_t[kMergeLanes][kMergeRows];
+  __shared__ double sl_s[kMergeLanes][kMergeRows], sl_t[kMergeLanes][kMergeRows], sa[kMergeLanes][kMergeRows];
+  const int r = threadIdx.x % kMergeRows, j = threadIdx.x / kMergeRows;
+  const int nv = ctrl->n_valid;
+  const int i = blockIdx.x * kMergeRows + r;
+  const bool live = i < nv;
   float ms = kNegBig, mt = kNegBig;
-  for (int k = 0; k < n_split; ++k) {
-    ms = fmaxf(ms, state[(long long)k * ld + i]);
-    mt = fmaxf(mt, state[2 * fs + (long long)k * ld + i]);
+  if (live)
+    for (int k = j; k < n_split; k += kMergeLanes) {
+      ms = fmaxf(ms, state[(long long)k * ld + i]);
+      mt = fmaxf(mt, state[2 * fs + (long long)k * ld + i]);
+    }
+  sm_s[j][r] = ms;
+  sm_t[j][r] = mt;
+  __syncthreads();
+  ms = kNegBig;
+  mt = kNegBig;
+  for (int q = 0; q < kMergeLanes; ++q) {
+    ms = fmaxf(ms, sm_s[q][r]);
+    mt = fmaxf(mt, sm_t[q][r]);
   }
   double ls = 0.0, lt = 0.0, a = 0.0;
-  for (int k = 0; k < n_split; ++k) {
-    const long long o = (long long)k * ld + i;
-    const double fs_ = exp2((double)state[o] - ms);
-    const double ft_ = exp2((double)state[2 * fs + o] - mt);
-    ls += state[fs + o] * fs_;
-    lt += state[3 * fs + o] * ft_;
-    if (kl_dir == 1) a += state[4 * fs + o] * fs_;
-    if (kl_dir == 2) a += state[4 * fs + o] * ft_;
+  if (live)
+    for (int k = j; k < n_split; k += kMergeLanes) {
+      const long long o = (long long)k * ld + i;
+      const double fs_ = exp2f(state[o] - ms);
+      const double ft_ = exp2f(state[2 * fs + o] - mt);
+      ls += state[fs + o] * fs_;
+      lt += state[3 * fs + o] * ft_;
+      if (kl_dir == 1) a += state[4 * fs + o] * fs_;
+      if (kl_dir == 2) a += state[4 * fs + o] * ft_;
+    }
+  sl_s[j][r] = ls;
+  sl_t[j][r] = lt;
+  sa[j][r] = a;
+  __syncthreads();
+  if (j != 0 || !live) return;
+  ls = lt = a = 0.0;
+  for (int q = 0; q < kMergeLanes; ++q) {
+    ls += sl_s[q][r];
+    lt += sl_t[q][r];
+    a += sa[q][r];
   }
   const double L2s = ms + log2(ls), L2t = mt + log2(lt);
-  const int r = idx[i];
-  lse_s[r] = float(L2s * 0.69314718055994530942);
-  lse_t[r] = float(L2t * 0.69314718055994530942);
+  const int row = idx[i];
+  lse_s[row] = float(L2s * 0.69314718055994530942);
+  lse_t[row] = float(L2t * 0.69314718055994530942);
   if (kl_dir == 1) {
     const float kl = float(0.69314718055994530942 * (a / ls - L2s + L2t));
-    loss_tok[r] = kl;
-    aux[r] = kl;
+    loss_tok[row] = kl;
+    aux[row] = kl;
   } else if (kl_dir == 2) {
     const float kl = float(0.69314718055994530942 * (a / lt - L2t + L2s));
-    loss_tok[r] = kl;
-    aux[r] = kl;
+    loss_tok[row] = kl;
+    aux[row] = kl;
   } else {
     row_l2s[i] = float(L2s);
     row_l2t[i] = float(L2t);
   }
 }
 
-// JSD: sum the per-split partial sums (base 2) and convert to nats.
-__global__ void jsd_finalize_kernel(const float* __restrict__ part, long long fs, int ld, int n_split,
-                                    const int* __restrict__ idx, const Ctrl* __restrict__ ctrl, float* loss_tok,
-                                    float* aux) {
-  const int i = blockIdx.x * blockDim.x + threadIdx.x;
-  if (i >= ctrl->n_valid) return;
+// JSD: sum the per-split partial sums (base 2) in a fixed order and convert to nats.
+__global__ void __launch_bounds__(kMergeRows * kMergeLanes)
+    jsd_finalize_kernel(const float* __restrict__ part, long long fs, int ld, int n_split,
+                        const int* __restrict__ idx, const Ctrl* __restrict__ ctrl, float* loss_tok, float* aux) {
+  __shared__ double sj[kMergeLanes][kMergeRows], sk[kMergeLanes][kMergeRows];
+  const int r = threadIdx.x % kMergeRows, j = threadIdx.x / kMergeRows;
+  const int nv = ctrl->n_valid;
+  const int i = blockIdx.x * kMergeRows + r;
+  const bool live = i < nv;
   double js = 0.0, ks = 0.0;
-  for (int k = 0; k < n_split; ++k) {
-    js += part[(long long)k * ld + i];
-    ks += part[fs + (long long)k * ld + i];
+  if (live)
+    for (int k = j; k < n_split; k += kMergeLanes) {
+      js += part[(long long)k * ld + i];
+      ks += part[fs + (long long)k * ld + i];
+    }
+  sj[j][r] = js;
+  sk[j][r] = ks;
+  __syncthreads();
+  if (j != 0 || !live) return;
+  js = ks = 0.0;
+  for (int q = 0; q < kMergeLanes; ++q) {
+    js += sj[q][r];
+    ks += sk[q][r];
   }
-  const int r = idx[i];
-  loss_tok[r] = float(js * 0.69314718055994530942);
-  aux[r] = float(ks * 0.69314718055994530942);
+  const int row = idx[i];
+  loss_tok[row] = float(js * 0.69314718055994530942);
+  aux[row] = float(ks * 0.69314718055994530942);
 }
 
 // Deterministic masked mean: fixed-order fp64 sum of loss_tok (masked rows hold 0).
@@ -185,7 +229,17 @@ __global__ void __launch_bounds__(1024) mean_kernel(const float* __restrict__ lo
   }
 }
 
-// Zero the dh_s rows of masked positions (valid rows are written by the first chunk).
+// dh_s[idx[i]] = dh_c[i] for the valid rows (the GEMMs accumulate into the compacted dh_c).
+__global__ void scatter_rows_kernel(const float* __restrict__ src, int d, float* __restrict__ dst,
+                                    const int* __restrict__ idx, const Ctrl* __restrict__ ctrl) {
+  const int i = blockIdx.x;
+  if (i >= ctrl->n_valid) return;
+  const float4* in = reinterpret_cast<const float4*>(src + (long long)i * d);
+  float4* out = reinterpret_cast<float4*>(dst + (long long)idx[i] * d);
+  for (int c = threadIdx.x; c < d / 4; c += blockDim.x) out[c] = in[c];
+}
+
+// Zero the dh_s rows of masked positions (valid rows are written by the scatter).
 __global__ void zero_masked_rows_kernel(const int64_t* __restrict__ labels, long long ignore_index, float* dh,
                                         int d) {
   const int r = blockIdx.x;

@@ -3,24 +3,31 @@
 // "Nitrobrew tweet analysis", section "Nitrobrew 的两个动作": for each vocabulary
 // block, z_s = h_s W_s[v0:v1]^T and z_t = h_t W_t[v0:v1]^T are formed, the online
 // softmax / log-sum-exp accumulators and the KL terms are updated, and the block is
-// discarded. Here one block is a 128-token x 256-column tile.
+// discarded. Here one block is a 256-token x 256-column tile computed by a pair of CTAs
+// (cta_group::2): each CTA stages 128 token rows of h and 128 vocabulary rows of W per K step
+// and holds its 128 rows of both fp32 accumulators.
 //
-// Tensor memory holds both fp32 accumulators of a tile (2 x 256 columns = all 512), so it
-// cannot be double-buffered. Instead the model with the larger K ("first") is multiplied
-// first; the epilogue copies the first accumulator into registers as soon as the tile is
-// complete and releases it, so the next tile's first-model MMAs run while the epilogue
-// streams the second accumulator. The second accumulator is released after its last read,
-// normally long before the next tile's first-model phase ends.
+// Tensor memory holds both accumulators of a tile (2 x 256 columns = all 512), so it cannot be
+// double-buffered. Instead the model with the larger K ("first") is multiplied first and
+// committed on its own barrier; the epilogue copies the first accumulator into registers while
+// the second model's MMAs run and releases it, so the next tile's first-model MMAs can start as
+// soon as the tile ends, while the epilogue streams the second accumulator (released after its
+// last read, normally long before the next tile's first-model phase ends).
 //
-// Warp roles (384 threads, one CTA per SM, persistent over work units):
-//   warp 0     TMA producer: 128 x 64 h tiles and 256 x 64 W tiles into a 4-stage ring
-//   warp 1     MMA issuer: 4 x tcgen05.mma 128x256x16 per K block; owns TMEM
+// Warp roles (384 threads per CTA, one CTA per SM, persistent over work units):
+//   warp 0     TMA producer (both CTAs): 128 x 64 h tile + 128 x 64 W tile per stage, 6 stages
+//   warp 1     MMA issuer (leader CTA only): 4 x tcgen05.mma 256x256x16 per K block; TMEM owner
 //   warps 2-3  idle (warpgroup 0 hands its registers to the epilogue: 56 vs 224 per thread)
 //   warps 4-11 epilogue: two warps per TMEM lane quarter, each thread one token row and one
 //              128-column half of the tile, base-2 online math in registers
 //
-// A work unit is (token tile, run of `tiles_per_unit` vocabulary tiles); each thread writes
-// its row's partial state once per unit (split = 2 * unit + column half).
+// Barriers: the leader's full[] barrier counts the TMA bytes of both CTAs; the MMA completion
+// is multicast to the empty[] / tfull[] barriers of both CTAs; the epilogue warps of both CTAs
+// arrive on the leader's tempty[]. Work ids come from the leader's TMA thread through a ring
+// mirrored into the peer CTA.
+//
+// A work unit is (256-row token tile, run of `tiles_per_unit` vocabulary tiles); each thread
+// writes its row's partial state once per unit (split = 2 * unit + column half).
 #pragma once
 
 #include "common.cuh"
@@ -29,12 +36,16 @@ namespace nbkl {
 
 struct SweepSmem {
   uint8_t* a;           // kStages x 16 KB
-  uint8_t* b;           // kStages x 32 KB
-  uint64_t* full;       // kStages
-  uint64_t* empty;      // kStages
-  uint64_t* tfull;      // tile complete (GEMM kernel: 2, one per accumulator stage)
-  uint64_t* tempty;     // accumulator released (sweep: [0] first model, [1] second model)
+  uint8_t* b;           // kStages x 16 KB
+  uint8_t* out;         // kEpiWarps x 4 KB TMA-store staging
+  uint64_t* full;       // kStages (leader: TMA bytes of both CTAs)
+  uint64_t* empty;      // kStages (both: MMA commit)
+  uint64_t* tfull;      // sweep: [1] first model, [0] whole tile complete; GEMM: one per stage
+  uint64_t* tempty;     // leader: accumulator released by all 16 epilogue warps of the pair
   uint64_t* drain;      // 1
+  uint64_t* ring_full;  // kRing: a work id was written to ring_slot (both CTAs)
+  uint64_t* ring_empty; // kRing: leader: every consumer of the pair has read it
+  int* ring_slot;       // kRing
   uint32_t* tmem_slot;
 };
 
@@ -43,13 +54,17 @@ __device__ __forceinline__ SweepSmem carve_smem(uint8_t* raw) {
   uint8_t* base = align1024(raw);
   s.a = base;
   s.b = base + kStages * kATileBytes;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(base + kStages * kStageBytes);
+  s.out = base + kStages * kStageBytes;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(s.out + kEpiWarps * kStageOutBytes);
   s.full = bars;
   s.empty = bars + kStages;
   s.tfull = bars + 2 * kStages;
   s.tempty = bars + 2 * kStages + 2;
   s.drain = bars + 2 * kStages + 4;
-  s.tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * kStages + 5);
+  s.ring_full = bars + 2 * kStages + 5;
+  s.ring_empty = s.ring_full + kRing;
+  s.ring_slot = reinterpret_cast<int*>(s.ring_empty + kRing);
+  s.tmem_slot = reinterpret_cast<uint32_t*>(s.ring_slot + kRing);
   return s;
 }
 
@@ -60,10 +75,47 @@ __device__ __forceinline__ void init_barriers(const SweepSmem& s) {
   }
   for (int i = 0; i < 2; ++i) {
     mbar_init(&s.tfull[i], 1);
-    mbar_init(&s.tempty[i], kEpiThreads);
+    mbar_init(&s.tempty[i], 2 * kEpiWarps);
   }
   mbar_init(s.drain, 1);
+  for (int i = 0; i < kRing; ++i) {
+    mbar_init(&s.ring_full[i], 1);
+    mbar_init(&s.ring_empty[i], kRingConsumers);
+  }
   fence_mbar_init();
+}
+
+// Common prologue of the pair kernels: barriers, TMEM (512 columns in each CTA), cluster sync.
+__device__ __forceinline__ uint32_t pair_prologue(const SweepSmem& s) {
+  const int warp = threadIdx.x / 32;
+  if (threadIdx.x == 0) init_barriers(s);
+  if (warp == 1) {
+    tmem_alloc_pair(smem_addr(s.tmem_slot), 512);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync_all();  // the peer's barriers exist before any cross-CTA arrive or TMA byte count
+  tc_fence_after();
+  return *s.tmem_slot;
+}
+
+__device__ __forceinline__ void pair_epilogue(const SweepSmem& s, uint32_t tmem_base, const WaitCtl& w) {
+  const int warp = threadIdx.x / 32;
+  tc_fence_before();
+  __syncthreads();
+  if (*reinterpret_cast<volatile int*>(w.status) != 0) {
+    // after a failure, give copies the peer may still have in flight time to land
+    const uint64_t t0 = global_timer_ns();
+    while (global_timer_ns() - t0 < 2000000ull) {
+    }
+  }
+  cluster_sync_all();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, 512);
+  }
 }
 
 struct UnitGrid {
@@ -73,14 +125,47 @@ struct UnitGrid {
 __device__ __forceinline__ UnitGrid unit_grid(const SweepArgs& p) {
   UnitGrid g;
   g.n_valid = *p.n_valid;
-  g.n_tt = (g.n_valid + kBlockM - 1) / kBlockM;
+  g.n_tt = (g.n_valid + kPairM - 1) / kPairM;
   g.n_vt = (p.v_end - p.v_begin + kBlockN - 1) / kBlockN;
   g.n_vu = (g.n_vt + p.tiles_per_unit - 1) / p.tiles_per_unit;
   g.n_units = g.n_tt * g.n_vu;
   return g;
 }
 
-// Bounded wait for the copies a failed producer may still have in flight.
+// ------------------------------------------------------------------ work distribution
+// The leader's TMA thread takes the next work id (from a global counter when `sched` is set,
+// so that pairs which start late, or share the GPU with another kernel, simply take fewer
+// items; else a static stride over pairs), writes it into the ring of both CTAs and arrives on
+// both ring_full[] barriers. The leader's MMA thread, the peer's TMA thread and the epilogue
+// warps of both CTAs read it and arrive on the leader's ring_empty[]. -1 ends the sequence.
+__device__ __forceinline__ int next_work(int* sched, int it) {
+  const int pair = int(blockIdx.x) >> 1, n_pairs = int(gridDim.x) >> 1;
+  return sched ? atomicAdd(sched, 1) : pair + it * n_pairs;
+}
+
+__device__ __forceinline__ bool ring_put(const SweepSmem& s, int it, int id, const WaitCtl& w) {
+  const int k = it % kRing;
+  if (!mbar_wait_cl(&s.ring_empty[k], ((it / kRing) & 1) ^ 1, w)) return false;
+  s.ring_slot[k] = id;
+  st_remote_u32(cluster_addr(smem_addr(&s.ring_slot[k]), 1), uint32_t(id));
+  mbar_arrive(&s.ring_full[k]);
+  mbar_arrive_remote(cluster_addr(smem_addr(&s.ring_full[k]), 1));
+  return true;
+}
+
+// `warp_wide`: every lane waits and reads, lane 0 arrives once for the warp.
+__device__ __forceinline__ bool ring_get(const SweepSmem& s, int it, int& id, const WaitCtl& w, bool warp_wide) {
+  const int k = it % kRing;
+  if (!mbar_wait_cl(&s.ring_full[k], (it / kRing) & 1, w)) return false;
+  id = *reinterpret_cast<volatile int*>(&s.ring_slot[k]);
+  if (warp_wide) __syncwarp();
+  if (!warp_wide || (threadIdx.x % 32) == 0)
+    mbar_arrive_remote(cluster_addr(smem_addr(&s.ring_empty[k]), 0));
+  return true;
+}
+
+// Bounded wait for the copies a failed producer may still have in flight (leader: its full[]
+// barriers count the bytes of both CTAs).
 __device__ __forceinline__ void drain_loads(const SweepSmem& s, const uint32_t* pend_stage,
                                             const uint32_t* pend_par, int n_issued) {
   const int n = min(n_issued, kStages);
@@ -93,18 +178,26 @@ __device__ __forceinline__ void drain_loads(const SweepSmem& s, const uint32_t* 
   }
 }
 
-// Bounded wait until every MMA this thread issued has completed.
+// Bounded wait until every pair MMA the leader issued has completed.
 __device__ __forceinline__ void drain_mma(const SweepSmem& s) {
-  umma_commit(smem_addr(s.drain));
+  umma_commit_pair_local(smem_addr(s.drain));
   const uint32_t a = smem_addr(s.drain);
   const uint64_t t0 = global_timer_ns();
   while (!mbar_test(a, 0) && global_timer_ns() - t0 < 100000000ull) {
   }
 }
 
-// ------------------------------------------------------------------ producer
+// Epilogue warp's release of a TMEM accumulator: after its own tcgen05.ld completed, lane 0
+// arrives on the leader's barrier.
+__device__ __forceinline__ void release_accumulator(uint64_t* bar) {
+  tc_fence_before();
+  __syncwarp();
+  if ((threadIdx.x % 32) == 0) mbar_arrive_remote(cluster_addr(smem_addr(bar), 0));
+}
+
+// ------------------------------------------------------------------ producer (both CTAs)
 __device__ __forceinline__ void sweep_producer(const SweepMaps& maps, const SweepArgs& p, const UnitGrid& g,
-                                               const SweepSmem& s, const WaitCtl& w) {
+                                               const SweepSmem& s, const WaitCtl& w, uint32_t rank) {
   int stage = 0;
   uint32_t phase = 0;
   uint32_t pend_stage[kStages], pend_par[kStages];
@@ -117,20 +210,31 @@ __device__ __forceinline__ void sweep_producer(const SweepMaps& maps, const Swee
   const int nk1 = p.teacher_first ? p.nkb_t : p.nkb_s, nk2 = p.teacher_first ? p.nkb_s : p.nkb_t;
   const int bm1 = p.teacher_first ? p.bmod_t : p.bmod_s, bm2 = p.teacher_first ? p.bmod_s : p.bmod_t;
   bool ok = true;
-  for (int u = blockIdx.x; u < g.n_units && ok; u += gridDim.x) {
+  for (int it = 0; ok; ++it) {
+    int u;
+    if (rank == 0) {
+      u = next_work(p.sched, it);
+      if (u >= g.n_units) u = -1;
+      if (!ring_put(s, it, u, w)) { ok = false; break; }
+    } else if (!ring_get(s, it, u, w, false)) {
+      ok = false;
+      break;
+    }
+    if (u < 0) break;
     const int vu = u / g.n_tt, tt = u % g.n_tt;
+    const int row0 = tt * kPairM + int(rank) * kBlockM;
     const int t_end = min((vu + 1) * p.tiles_per_unit, g.n_vt);
     for (int t = vu * p.tiles_per_unit; t < t_end && ok; ++t) {
-      const int v0 = p.v_begin + t * kBlockN;
+      const int v0 = p.v_begin + t * kBlockN + int(rank) * kHalfB;
       for (int kb = 0; kb < nk1 + nk2; ++kb) {
-        if (!mbar_wait(&s.empty[stage], phase ^ 1u, w)) { ok = false; break; }
+        if (!mbar_wait_cl(&s.empty[stage], phase ^ 1u, w)) { ok = false; break; }
         const bool one = kb < nk1;
         const int k = one ? kb : kb - nk1;
         const int kbb = k % (one ? bm1 : bm2);
         const uint32_t bar = smem_addr(&s.full[stage]);
-        mbar_arrive_expect_tx(&s.full[stage], kStageBytes);
-        tma_load_2d(smem_addr(s.a + stage * kATileBytes), one ? a1 : a2, bar, k * kBlockK, tt * kBlockM);
-        tma_load_2d(smem_addr(s.b + stage * kBTileBytes), one ? b1 : b2, bar, kbb * kBlockK, v0);
+        if (rank == 0) mbar_arrive_expect_tx(&s.full[stage], kPairStageBytes);
+        tma_load_2d_pair(smem_addr(s.a + stage * kATileBytes), one ? a1 : a2, bar, k * kBlockK, row0);
+        tma_load_2d_pair(smem_addr(s.b + stage * kBTileBytes), one ? b1 : b2, bar, kbb * kBlockK, v0);
         pend_stage[n_issued % kStages] = stage;
         pend_par[n_issued % kStages] = phase;
         ++n_issued;
@@ -138,18 +242,21 @@ __device__ __forceinline__ void sweep_producer(const SweepMaps& maps, const Swee
       }
     }
   }
-  if (!ok) drain_loads(s, pend_stage, pend_par, n_issued);
+  if (!ok && rank == 0) drain_loads(s, pend_stage, pend_par, n_issued);
 }
 
-// ------------------------------------------------------------------ MMA issuer
+// ------------------------------------------------------------------ MMA issuer (leader)
 __device__ __forceinline__ void sweep_mma(const SweepArgs& p, const UnitGrid& g, const SweepSmem& s,
                                           uint32_t tmem_base, const WaitCtl& w) {
   int stage = 0;
   uint32_t phase = 0;
-  uint32_t lt = 0;  // tiles processed by this CTA
+  uint32_t lt = 0;  // tiles processed by this pair
   const int nk1 = p.teacher_first ? p.nkb_t : p.nkb_s, nk2 = p.teacher_first ? p.nkb_s : p.nkb_t;
   bool ok = true;
-  for (int u = blockIdx.x; u < g.n_units && ok; u += gridDim.x) {
+  for (int it = 0; ok; ++it) {
+    int u;
+    if (!ring_get(s, it, u, w, false)) { ok = false; break; }
+    if (u < 0) break;
     const int vu = u / g.n_tt;
     const int t_end = min((vu + 1) * p.tiles_per_unit, g.n_vt);
     for (int t = vu * p.tiles_per_unit; t < t_end && ok; ++t, ++lt) {
@@ -157,8 +264,8 @@ __device__ __forceinline__ void sweep_mma(const SweepArgs& p, const UnitGrid& g,
         const bool one = kb < nk1;
         const int k = one ? kb : kb - nk1;
         if (k == 0) {
-          // the accumulator of this model must have been read by the epilogue
-          if (!mbar_wait(&s.tempty[one ? 0 : 1], (lt & 1u) ^ 1u, w)) { ok = false; break; }
+          // the accumulator of this model must have been read by both CTAs' epilogues
+          if (!mbar_wait_cl(&s.tempty[one ? 0 : 1], (lt & 1u) ^ 1u, w)) { ok = false; break; }
           tc_fence_after();
         }
         if (!mbar_wait(&s.full[stage], phase, w)) { ok = false; break; }
@@ -168,14 +275,16 @@ __device__ __forceinline__ void sweep_mma(const SweepArgs& p, const UnitGrid& g,
         const uint32_t sb = smem_addr(s.b + stage * kBTileBytes);
 #pragma unroll
         for (int j = 0; j < kBlockK / 16; ++j) {
-          umma_bf16(d, make_sdesc(sa + j * 32, 16, 1024), make_sdesc(sb + j * 32, 16, 1024), kIdescKK,
-                    (k > 0 || j > 0) ? 1u : 0u);
+          umma_bf16_pair(d, make_sdesc(sa + j * 32, 16, 1024), make_sdesc(sb + j * 32, 16, 1024), kIdescKK,
+                         (k > 0 || j > 0) ? 1u : 0u);
         }
-        umma_commit(smem_addr(&s.empty[stage]));
+        umma_commit_pair_both(smem_addr(&s.empty[stage]));
         if (++stage == kStages) { stage = 0; phase ^= 1u; }
+        // first accumulator complete: the epilogues copy it out while the second model runs
+        if (kb == nk1 - 1) umma_commit_pair_both(smem_addr(&s.tfull[1]));
       }
       if (!ok) break;
-      umma_commit(smem_addr(&s.tfull[0]));
+      umma_commit_pair_both(smem_addr(&s.tfull[0]));
     }
   }
   if (!ok) drain_mma(s);
@@ -266,9 +375,12 @@ __device__ __forceinline__ float grad_elem(float xs, float xt, const RowConst& c
   return c.omb * S * fmaf(kLn2, ys - ym, -c.aux);
 }
 
+// Gradient of one 32-column chunk of a row, packed to bf16 and written into the warp's
+// staging buffer (32 rows x 64 bytes, 64-byte swizzle: 16-byte piece c of row r sits at piece
+// c ^ ((r >> 1) & 3)), from where one TMA store per warp writes the 32 x 32 block.
 template <int MODE, bool MASKED>
 __device__ __forceinline__ void chunk_grad(const float (&zs)[32], const float (&zt)[32], int n_ok, float scale,
-                                           const RowConst& c, float gs, __nv_bfloat16* dst) {
+                                           const RowConst& c, float gs, uint8_t* stage_row, int r) {
   uint32_t packed[16];
 #pragma unroll
   for (int j = 0; j < 32; j += 2) {
@@ -279,16 +391,16 @@ __device__ __forceinline__ void chunk_grad(const float (&zs)[32], const float (&
     __nv_bfloat162 h = __floats2bfloat162_rn(g0, g1);
     packed[j / 2] = *reinterpret_cast<uint32_t*>(&h);
   }
-  uint4* d4 = reinterpret_cast<uint4*>(dst);
 #pragma unroll
   for (int q = 0; q < 4; ++q)
-    d4[q] = make_uint4(packed[4 * q], packed[4 * q + 1], packed[4 * q + 2], packed[4 * q + 3]);
+    *reinterpret_cast<uint4*>(stage_row + ((q ^ ((r >> 1) & 3)) * 16)) =
+        make_uint4(packed[4 * q], packed[4 * q + 1], packed[4 * q + 2], packed[4 * q + 3]);
 }
 
 template <int MODE>
 __device__ __forceinline__ void process_chunk(float (&zs)[32], float (&zt)[32], int n_ok, const SweepArgs& p,
                                               const RowConst& c, float gs, RowState& r, float& js, float& ks,
-                                              __nv_bfloat16* gdst) {
+                                              uint8_t* gstage, int lane) {
   const bool masked = n_ok < 32;
   if (MODE <= kStateT) {
     if (masked) chunk_state<MODE, true>(zs, zt, n_ok, p.scale, r);
@@ -297,20 +409,24 @@ __device__ __forceinline__ void process_chunk(float (&zs)[32], float (&zt)[32], 
     if (masked) chunk_jsd<true>(zs, zt, n_ok, p.scale, c, js, ks);
     else chunk_jsd<false>(zs, zt, n_ok, p.scale, c, js, ks);
   } else {
-    if (masked) chunk_grad<MODE, true>(zs, zt, n_ok, p.scale, c, gs, gdst);
-    else chunk_grad<MODE, false>(zs, zt, n_ok, p.scale, c, gs, gdst);
+    if (masked) chunk_grad<MODE, true>(zs, zt, n_ok, p.scale, c, gs, gstage, lane);
+    else chunk_grad<MODE, false>(zs, zt, n_ok, p.scale, c, gs, gstage, lane);
   }
 }
 
 // ------------------------------------------------------------------ epilogue
 template <int MODE>
-__device__ __forceinline__ void sweep_epilogue(const SweepArgs& p, const UnitGrid& g, const SweepSmem& s,
-                                               uint32_t tmem_base, const WaitCtl& w) {
+__device__ __forceinline__ void sweep_epilogue(const SweepMaps& maps, const SweepArgs& p, const UnitGrid& g,
+                                               const SweepSmem& s, uint32_t tmem_base, const WaitCtl& w) {
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int q = warp & 3;                      // TMEM lane quarter this warp may access
   const int half = (warp - kEpiWarp0) >> 2;    // column half of the tile
   const int row_in_tile = q * 32 + lane;
   const uint32_t lane_addr = uint32_t(q * 32) << 16;
+  const uint32_t rank = cluster_rank();
+  uint8_t* stage = s.out + (warp - kEpiWarp0) * kStageOutBytes;
+  uint8_t* stage_row = stage + lane * 64;
+  bool staged = false;                                           // a TMA store may still read it
   const uint32_t col1 = tmem_base + lane_addr + half * kHalfN;   // first model
   const uint32_t col2 = col1 + kBlockN;                          // second model
   uint32_t lt = 0;
@@ -321,9 +437,12 @@ __device__ __forceinline__ void sweep_epilogue(const SweepArgs& p, const UnitGri
   c.lg2_b = p.lg2_b;
   const float gscale = (MODE >= kGradFkl) ? *p.gscale : 0.f;
 
-  for (int u = blockIdx.x; u < g.n_units; u += gridDim.x) {
+  for (int it = 0;; ++it) {
+    int u;
+    if (!ring_get(s, it, u, w, true)) return;
+    if (u < 0) break;
     const int vu = u / g.n_tt, tt = u % g.n_tt;
-    const int row = tt * kBlockM + row_in_tile;
+    const int row = tt * kPairM + int(rank) * kBlockM + row_in_tile;
     const bool row_ok = row < g.n_valid;
     if (MODE >= kJsd) {
       c.l2s = p.row_l2s[row];
@@ -336,28 +455,38 @@ __device__ __forceinline__ void sweep_epilogue(const SweepArgs& p, const UnitGri
     const int t_end = min((vu + 1) * p.tiles_per_unit, g.n_vt);
     for (int t = vu * p.tiles_per_unit; t < t_end; ++t, ++lt) {
       const int v0 = p.v_begin + t * kBlockN + half * kHalfN;
-      if (!mbar_wait(&s.tfull[0], lt & 1u, w)) return;
+      if (!mbar_wait_cl(&s.tfull[1], lt & 1u, w)) return;   // first model complete
       tc_fence_after();
       float F[4][32];
 #pragma unroll
       for (int ch = 0; ch < 4; ++ch) tmem_ld32(col1 + ch * 32, F[ch]);
       tmem_wait_ld();
-      tc_fence_before();
-      mbar_arrive(&s.tempty[0]);
+      release_accumulator(&s.tempty[0]);
+      if (!mbar_wait_cl(&s.tfull[0], lt & 1u, w)) return;   // second model complete
+      tc_fence_after();
 #pragma unroll
       for (int ch = 0; ch < 4; ++ch) {
         float C[32];
         tmem_ld32(col2 + ch * 32, C);
         tmem_wait_ld();
-        if (ch == 3) {
-          tc_fence_before();
-          mbar_arrive(&s.tempty[1]);
-        }
+        if (ch == 3) release_accumulator(&s.tempty[1]);
         const int c0 = v0 + ch * 32;
         const int n_ok = p.V - c0;            // columns of this chunk inside the vocabulary
-        __nv_bfloat16* gdst = (MODE >= kGradFkl) ? p.G + (long long)row * p.ldG + (c0 - p.v_begin) : nullptr;
-        if (p.teacher_first) process_chunk<MODE>(C, F[ch], n_ok, p, c, gs, r, js, ks, gdst);
-        else process_chunk<MODE>(F[ch], C, n_ok, p, c, gs, r, js, ks, gdst);
+        if (MODE >= kGradFkl) {
+          if (staged && lane == 0) bulk_wait_read();
+          __syncwarp();
+        }
+        if (p.teacher_first) process_chunk<MODE>(C, F[ch], n_ok, p, c, gs, r, js, ks, stage_row, lane);
+        else process_chunk<MODE>(F[ch], C, n_ok, p, c, gs, r, js, ks, stage_row, lane);
+        if (MODE >= kGradFkl) {
+          fence_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_2d(&maps.g_out, smem_addr(stage), c0 - p.v_begin, row - lane);
+            bulk_commit();
+          }
+          staged = true;
+        }
       }
     }
     const long long off = (long long)(2 * vu + half) * p.ld + row;
@@ -372,47 +501,36 @@ __device__ __forceinline__ void sweep_epilogue(const SweepArgs& p, const UnitGri
       p.out[p.field_stride + off] = ks;
     }
   }
+  if (MODE >= kGradFkl && lane == 0) bulk_wait_all();
 }
 
 template <int MODE>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     sweep_kernel(const __grid_constant__ SweepMaps maps, const SweepArgs p) {
   extern __shared__ uint8_t smem_raw[];
   const SweepSmem s = carve_smem(smem_raw);
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  if (threadIdx.x == 0) init_barriers(s);
+  const uint32_t rank = cluster_rank();
   if (warp == 0 && lane == 0) {
     tma_prefetch_map(&maps.a_s);
     tma_prefetch_map(&maps.b_s);
     tma_prefetch_map(&maps.a_t);
     tma_prefetch_map(&maps.b_t);
+    if (MODE >= kGradFkl) tma_prefetch_map(&maps.g_out);
   }
-  if (warp == 1) {
-    tmem_alloc(smem_addr(s.tmem_slot), 512);
-    tmem_relinquish();
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem_base = *s.tmem_slot;
+  const uint32_t tmem_base = pair_prologue(s);
   const UnitGrid g = unit_grid(p);
   const WaitCtl w{p.status, p.wait_limit_ns};
 
   if (warp < kEpiWarp0) {
     regs_shrink<kRegsCtl>();
-    if (warp == 0 && lane == 0) sweep_producer(maps, p, g, s, w);
-    if (warp == 1 && lane == 0) sweep_mma(p, g, s, tmem_base, w);
+    if (warp == 0 && lane == 0) sweep_producer(maps, p, g, s, w, rank);
+    if (warp == 1 && lane == 0 && rank == 0) sweep_mma(p, g, s, tmem_base, w);
   } else {
     regs_grow<kRegsEpi>();
-    sweep_epilogue<MODE>(p, g, s, tmem_base, w);
+    sweep_epilogue<MODE>(maps, p, g, s, tmem_base, w);
   }
-  tc_fence_before();
-  __syncthreads();
-  if (warp == 1) {
-    __syncwarp();
-    tc_fence_after();
-    tmem_dealloc(tmem_base, 512);
-  }
+  pair_epilogue(s, tmem_base, w);
 }
 
 }  // namespace nbkl

@@ -100,12 +100,14 @@ WORKLOADS = {
 
 
 # Same widths and statistics as a named workload but fewer tokens and a smaller vocabulary,
-# so that a detailed profiler capture of one kernel stays small (inputs still exceed L2).
+# so that a detailed profiler capture of one kernel stays small (the unembeddings, 543 MB,
+# still exceed L2). 512 valid rows (4 token tiles) x 37 units of 2048 columns = 148 forward
+# units: one per SM, so the capture shows steady-state behaviour, not a ragged last wave.
 PROFILE_WORKLOADS = {
     "opd_0p6b_4b_prof": Workload(
-        "opd_0p6b_4b_prof", 1, 2048, 1024, 2560, 32768, 1.0, 1.0, 3.0,
-        teacher="correlated", mask="prefix", masked_per_seq=819,
-        description="profiling size of opd_0p6b_4b: 2048 tokens, V 32768"),
+        "opd_0p6b_4b_prof", 1, 640, 1024, 2560, 75776, 1.0, 1.0, 3.0,
+        teacher="correlated", mask="prefix", masked_per_seq=128,
+        description="profiling size of opd_0p6b_4b: 640 tokens (512 valid), V 75776"),
 }
 
 
