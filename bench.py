@@ -169,18 +169,21 @@ def blas_threads():
     return len(os.sched_getaffinity(0))
 
 
-def cpu_baseline(x, budget_s=15.0):
+def cpu_baseline(x, min_s=10.0, max_positions=None):
+    """Oracle throughput on random positions of the workload: the sample doubles until one
+    timed run takes at least `min_s` seconds (the oracle has a large fixed cost per call)."""
     rng = np.random.default_rng(7)
     N = x.labels.shape[0]
-    t0 = time.perf_counter()
-    first = np.sort(rng.choice(N, size=64, replace=False))
-    oracle_sample_run(x, first)
-    t1 = time.perf_counter() - t0
-    n = int(min(N, max(64, 64 * (budget_s / max(t1, 1e-3)))))
-    pos = np.sort(rng.choice(N, size=n, replace=False))
-    t0 = time.perf_counter()
-    oracle_sample_run(x, pos)
-    dt = time.perf_counter() - t0
+    cap = N if max_positions is None else min(N, max_positions)
+    n = min(64, cap)
+    while True:
+        pos = np.sort(rng.choice(N, size=n, replace=False))
+        t0 = time.perf_counter()
+        oracle_sample_run(x, pos)
+        dt = time.perf_counter() - t0
+        if dt >= min_s or n >= cap:
+            break
+        n = min(cap, 2 * n)
     nv = int((x.labels[pos] != -100).sum())
     return {"value": n / dt, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
             "sample": f"{n} of {N} positions ({nv} valid) of workload {x.workload.name}, "
@@ -220,6 +223,22 @@ def run_reference(args):
     }
     print(json.dumps(line), flush=True)
     return 0
+
+
+def max_over_ranks(value: float, world: int, device) -> float:
+    """Maximum of a per-rank scalar (elapsed ms) over the process group."""
+    if world <= 1:
+        return float(value)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(units_per_rank: int, world: int, ms_per_step: float) -> float:
+    """Units of all ranks per second (every rank runs its own replica of the step)."""
+    return units_per_rank * world / (ms_per_step * 1e-3)
 
 
 def workload_config(w, n_valid, world):
@@ -306,11 +325,7 @@ def run_library(args):
     cnt_arr = (ctypes.c_int * 5)()
     lib.nb_kl_timing_read(ctypes.cast(ms_arr, ctypes.c_void_p), ctypes.cast(cnt_arr, ctypes.c_void_p), 5)
     clk = clocks.stop() if rank == 0 else None
-    ms = e0.elapsed_time(e1)
-    if world > 1:
-        t = torch.tensor([ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
     peak_extra = torch.cuda.max_memory_allocated(dev) - mem0
 
     # ---- end-to-end through the public API with host buffers
@@ -342,17 +357,13 @@ def run_library(args):
         e2e_step()
     e3.record(stream)
     barrier()
-    ms_e2e = e2.elapsed_time(e3)
-    if world > 1:
-        t = torch.tensor([ms_e2e], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_e2e = float(t.item())
+    ms_e2e = max_over_ranks(e2.elapsed_time(e3), world, dev)
 
     result = None
     if rank == 0:
         ms_step = ms / args.steps
         tokens = N * world
-        value = tokens / (ms_step * 1e-3)
+        value = whole_job_rate(N, world, ms_step)
         flops = algorithmic_flops(w, n_valid)
         step_flops = sum(flops.values())
         tflops = step_flops / (ms_step * 1e-3) / 1e12
@@ -378,7 +389,7 @@ def run_library(args):
                          "frac": achieved / peak, "traffic": traffic,
                          "algorithmic_flops_per_launch": per_launch_flops, "launch_ms": per_launch_ms},
             "kernel_ms_per_step": kms, "kernel_launches_per_step": kcount,
-            "e2e": {"value": tokens / (ms_e2e / e2e_steps * 1e-3), "unit": "tokens/s",
+            "e2e": {"value": whole_job_rate(N, world, ms_e2e / e2e_steps), "unit": "tokens/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps},
             "gpu_launches": launches,
             "clocks": clk,

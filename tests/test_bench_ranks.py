@@ -1,0 +1,50 @@
+"""Host logic of the multi-rank benchmark, on CPU with a world-size-2 gloo group: every rank
+runs its own replica, the elapsed time is the maximum over ranks, the rate counts all ranks'
+tokens, and the reference arm does its work on rank 0 only."""
+
+import os
+import socket
+
+import pytest
+import torch.multiprocessing as mp
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _worker(rank, world, port, out):
+    import torch.distributed as dist
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world),
+                      LOCAL_RANK=str(rank))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    import bench
+    r, w, lr = bench.dist_env()
+    ms = bench.max_over_ranks(10.0 + 5.0 * rank, w, "cpu")
+    rate = bench.whole_job_rate(8192, w, ms)
+    out[rank] = (r, w, lr, ms, rate)
+    dist.barrier()
+    dist.destroy_process_group()
+
+
+def test_two_rank_timing_and_rate():
+    port = _free_port()
+    mgr = mp.get_context("spawn").Manager()
+    out = mgr.dict()
+    mp.start_processes(_worker, args=(2, port, out), nprocs=2, join=True, start_method="spawn")
+    assert out[0][:3] == (0, 2, 0) and out[1][:3] == (1, 2, 1)
+    for r in (0, 1):
+        assert out[r][3] == 15.0                       # max over ranks
+        assert out[r][4] == pytest.approx(2 * 8192 / 0.015)
+
+
+def test_reference_arm_runs_on_rank0_only(monkeypatch, capsys):
+    import argparse
+    import bench
+    monkeypatch.setenv("RANK", "1")
+    monkeypatch.setenv("WORLD_SIZE", "2")
+    args = argparse.Namespace(workload="tiny", steps=3, warmup=3)
+    assert bench.run_reference(args) == 0
+    assert capsys.readouterr().out == ""
