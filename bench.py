@@ -83,13 +83,14 @@ def kernel_source_sha():
 
 
 def profiled_traffic(kernel: str, workload: str):
-    """Per-launch DRAM bytes from a committed ncu summary, if it matches the current source."""
-    p = os.path.join(ROOT, "profiles", f"{kernel}_{workload}.md")
+    """Per-launch DRAM bytes (read + write) of `kernel` from the committed full-size ncu summary
+    of the workload, if that summary was taken from the current device code."""
+    p = os.path.join(ROOT, "profiles", f"fullsize_{workload}.md")
     if not os.path.exists(p):
         return None
     txt = open(p).read()
     m_sha = re.search(r"kernel_source_sha:\s*([0-9a-f]+)", txt)
-    m_tr = re.search(r"dram_bytes_per_launch:\s*([0-9.eE+]+)", txt)
+    m_tr = re.search(re.escape(kernel) + r"\.dram_bytes_per_launch:\s*([0-9.eE+]+)", txt)
     if not m_sha or not m_tr or m_sha.group(1) != kernel_source_sha():
         return None
     return float(m_tr.group(1))
@@ -389,6 +390,8 @@ def run_library(args):
                          "frac": achieved / peak, "traffic": traffic,
                          "algorithmic_flops_per_launch": per_launch_flops, "launch_ms": per_launch_ms},
             "kernel_ms_per_step": kms, "kernel_launches_per_step": kcount,
+            "kernel_tflops": {c: (flops[c] / (kms[c] * 1e-3) / 1e12 if kms[c] > 0 else None)
+                              for c in ("sweep_fwd", "sweep_jsd", "sweep_grad", "gemm_bwd")},
             "e2e": {"value": whole_job_rate(N, world, ms_e2e / e2e_steps), "unit": "tokens/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps},
             "gpu_launches": launches,
