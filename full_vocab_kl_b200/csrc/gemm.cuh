@@ -132,8 +132,8 @@ __device__ __forceinline__ void gemm_mma(const GemmArgs& p, int nv, const SweepS
     tc_fence_after();
     const uint32_t d = tmem_base + acc * kBlockN;
     for (int kb = 0; kb < ti.nkb; ++kb) {
+      // TMA bytes are ordered by the barrier's transaction count: no tcgen05 fence here
       if (!mbar_wait(&s.full[stage], phase, w)) { ok = false; break; }
-      tc_fence_after();
       const uint32_t sa = smem_addr(s.a + stage * kATileBytes);
       const uint32_t sb = smem_addr(s.b + stage * kBTileBytes);
 #pragma unroll

@@ -92,11 +92,12 @@ bool make_layout(const nb_kl_shape* sh, float beta, Layout& L) {
   L.lda_t = int64_t(L.kb_t) * kBlockK * (L.split ? 2 : 1);
   L.n_vt = int((L.V + kBlockN - 1) / kBlockN);
   L.n_split = 2 * ((L.n_vt + kTilesPerUnitFwd - 1) / kTilesPerUnitFwd);  // two column halves per unit
-  // default chunk: about 4096 gradient tiles per sweep launch (so the two gradient buffers
-  // take ~0.5 GB whatever the token count), between 2048 and 32768 columns
-  const int64_t auto_chunk = round_up(std::max<int64_t>(2048, std::min<int64_t>(32768, (int64_t(1) << 20) /
-                                                                                    (L.N_pad / kBlockM))),
-                                      kBlockN);  // 128-row halves of the pair tiles
+  // default chunk: about 4096 gradient tiles per sweep launch (the two gradient buffers then
+  // take ~0.5 GB whatever the token count), but at least 4 d_s columns so that the compacted
+  // dh accumulator is not re-added too often; between 2048 and 32768 columns
+  const int64_t by_tiles = (int64_t(1) << 20) / (L.N_pad / kBlockM);
+  const int64_t auto_chunk =
+      round_up(std::max<int64_t>(2048, std::min<int64_t>(32768, std::max<int64_t>(by_tiles, 4 * L.d_s))), kBlockN);
   L.chunk_v = sh->chunk_v ? sh->chunk_v : std::min<int64_t>(auto_chunk, round_up(L.V, kBlockN));
   const bool jsd = beta > 0.f && beta < 1.f;
   size_t off = kCtrlBytes;

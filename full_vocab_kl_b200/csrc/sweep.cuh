@@ -268,8 +268,8 @@ __device__ __forceinline__ void sweep_mma(const SweepArgs& p, const UnitGrid& g,
           if (!mbar_wait_cl(&s.tempty[one ? 0 : 1], (lt & 1u) ^ 1u, w)) { ok = false; break; }
           tc_fence_after();
         }
+        // TMA bytes are ordered by the barrier's transaction count: no tcgen05 fence here
         if (!mbar_wait(&s.full[stage], phase, w)) { ok = false; break; }
-        tc_fence_after();
         const uint32_t d = tmem_base + (one ? 0 : kBlockN);
         const uint32_t sa = smem_addr(s.a + stage * kATileBytes);
         const uint32_t sb = smem_addr(s.b + stage * kBTileBytes);
