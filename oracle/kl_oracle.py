@@ -37,6 +37,17 @@ Readings where the pages leave a step open (each is listed in the design notes):
    probability, so ``0 * log 0`` never arises; a probability that underflows to
    0 contributes 0.
 8. Rows are not shifted: row n of h_s, h_t and labels is one position.
+
+Per-token side outputs of the student (``forward(..., side=True)``), from
+"01 · 论文精读与参考实现全景映射" (ars-opd-rebuild docs), section 1 (Eq. 6,
+the per-token entropy H_t that the peak-entropy scheduler ranks; Eq. 8, the
+log-probability the student gives its own sampled token) and section 3.5:
+
+9. Both are taken under the same tempered student distribution S = softmax(z_s / tau)
+   that the loss uses (at tau = 1, the model's own distribution):
+   ``entropy_s = -sum_v S log S`` and ``logp_label = log S[label]`` in nats.
+10. The sampled token of row n is ``labels[n]`` (rows are not shifted, reading 8);
+    masked rows get 0 for both; a label outside [0, V) gets NaN log-probability.
 """
 
 from __future__ import annotations
@@ -116,6 +127,17 @@ def dloss_du_student(logS: np.ndarray, logT: np.ndarray, beta: float, loss: np.n
     return (1.0 - beta) * S * (logS - logM - aux[:, None])
 
 
+def student_side_rows(logS: np.ndarray, labels: np.ndarray):
+    """Entropy -sum S log S and log S[label] for a block of rows (readings 9 and 10)."""
+    H = -(np.exp(logS) * logS).sum(axis=1)
+    V = logS.shape[1]
+    lab = np.asarray(labels, dtype=np.int64)
+    inside = (lab >= 0) & (lab < V)
+    logp = np.full(lab.shape[0], np.nan)
+    logp[inside] = logS[np.flatnonzero(inside), lab[inside]]
+    return H, logp
+
+
 def _check(beta: float, tau: float):
     if not (0.0 <= beta <= 1.0):
         raise ValueError("beta must be in [0, 1]")
@@ -130,12 +152,14 @@ def _row_blocks(rows: np.ndarray, block: int):
 
 def forward(h_s, W_s, h_t, W_t, labels, beta: float, tau: float, *,
             rows: Optional[Sequence[int]] = None, ignore_index: int = IGNORE_INDEX,
-            row_block: int = 256) -> dict:
+            row_block: int = 256, side: bool = False) -> dict:
     """Per-token loss, both LSEs, aux, and the per-token mean.
 
     ``rows`` restricts the per-token outputs to those positions (the mean is then
     only returned when every valid row is among them). Returns float64 arrays of
-    length N (zeros where not computed or masked).
+    length N (zeros where not computed or masked). With ``side`` the student's
+    per-token entropy and sampled-token log-probability are added
+    (``entropy_s``, ``logp_label``).
     """
     _check(beta, tau)
     labels = np.asarray(labels)
@@ -144,13 +168,16 @@ def forward(h_s, W_s, h_t, W_t, labels, beta: float, tau: float, *,
     n_valid = int(valid.sum())
     todo = np.flatnonzero(valid) if rows is None else np.asarray(
         [r for r in rows if valid[r]], dtype=np.int64)
-    out = {k: np.zeros(N) for k in ("loss_tok", "lse_s", "lse_t", "aux")}
+    keys = ("loss_tok", "lse_s", "lse_t", "aux") + (("entropy_s", "logp_label") if side else ())
+    out = {k: np.zeros(N) for k in keys}
     for r in _row_blocks(todo, row_block):
         logS, lse_s = log_softmax(tempered_logits(h_s[r], W_s, tau))
         logT, lse_t = log_softmax(tempered_logits(h_t[r], W_t, tau))
         loss, aux = divergence_rows(logS, logT, beta)
         out["loss_tok"][r], out["aux"][r] = loss, aux
         out["lse_s"][r], out["lse_t"][r] = lse_s, lse_t
+        if side:
+            out["entropy_s"][r], out["logp_label"][r] = student_side_rows(logS, labels[r])
     complete = len(todo) == n_valid
     out["n_valid"] = n_valid
     if not complete:

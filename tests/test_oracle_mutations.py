@@ -104,3 +104,44 @@ def test_lse_missing_log_caught(monkeypatch):
 
     monkeypatch.setattr(ko, "log_softmax", bad)
     assert _fails(pins.test_lse_zero_weights_is_log_v)
+
+
+# ------------------------------------------------------------------ side outputs
+import test_oracle_side_pins as side_pins  # noqa: E402
+
+
+def _side_mutant(monkeypatch, fn):
+    orig = ko.student_side_rows
+    monkeypatch.setattr(ko, "student_side_rows", lambda lS, lab: fn(orig, lS, lab))
+
+
+def test_entropy_sign_slip_caught(monkeypatch):
+    _side_mutant(monkeypatch, lambda o, lS, lab: (-o(lS, lab)[0], o(lS, lab)[1]))
+    assert _fails(side_pins.test_uniform_student)
+
+
+def test_entropy_in_bits_caught(monkeypatch):
+    _side_mutant(monkeypatch, lambda o, lS, lab: (o(lS, lab)[0] / math.log(2.0), o(lS, lab)[1]))
+    assert _fails(side_pins.test_two_level_closed_form, 3, 2.0, -1.0, 2.0)
+
+
+def test_label_off_by_one_caught(monkeypatch):
+    _side_mutant(monkeypatch, lambda o, lS, lab: o(lS, np.minimum(np.asarray(lab) + 1, lS.shape[1] - 1)))
+    assert _fails(side_pins.test_brute_force_tiny, 1.0, 12)
+
+
+def test_logp_without_normaliser_caught(monkeypatch):
+    # log-probabilities read from the tempered logits themselves (u instead of u - lse)
+    def raw(u):
+        m = u.max(axis=1, keepdims=True)
+        lse = m + np.log(np.exp(u - m).sum(axis=1, keepdims=True))
+        return u, lse[:, 0]
+
+    monkeypatch.setattr(ko, "log_softmax", raw)
+    assert _fails(side_pins.test_two_level_closed_form, 3, 2.0, -1.0, 2.0)
+
+
+def test_untempered_side_outputs_caught(monkeypatch):
+    # at tau = 2: logS * 2 re-normalised is the softmax of z itself
+    _side_mutant(monkeypatch, lambda o, lS, lab: o(ko.log_softmax(lS * 2.0)[0], lab))
+    assert _fails(side_pins.test_two_level_closed_form, 3, 2.0, -1.0, 2.0)
