@@ -72,11 +72,15 @@ def algorithmic_flops(w, n_valid):
     }
 
 
+# headers that define the profiled tensor-core kernels (the vocabulary sweep and the GEMM)
+PROFILED_SOURCES = ("common.cuh", "gemm.cuh", "ptx.cuh", "sweep.cuh")
+
+
 def kernel_source_sha():
-    """Hash of the device-code headers: a profile summary is only used while it matches."""
+    """Hash of the sweep and GEMM device code: a profile summary is only used while it matches."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "full_vocab_kl_b200", "csrc")
-    for name in sorted(n for n in os.listdir(csrc) if n.endswith(".cuh")):
+    for name in PROFILED_SOURCES:
         with open(os.path.join(csrc, name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]

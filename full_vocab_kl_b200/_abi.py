@@ -22,6 +22,7 @@ NB_ERR_TIMEOUT = -5
 NB_BF16 = 0
 NB_F32 = 1
 NOALLOC_SCRATCH_BYTES = 64 * 1024 * 1024
+VP_FIELDS = 7   # NB_KL_VP_FIELDS: floats per token of a vocabulary shard's state
 
 # every function the header declares, with (restype, argtypes)
 SIGNATURES = {
@@ -29,6 +30,17 @@ SIGNATURES = {
     "nb_kl_forward": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_float, c_float,
                               c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_size_t,
                               c_void_p]),
+    "nb_kl_forward_side": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_float, c_float,
+                                   c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
+                                   c_void_p, c_size_t, c_void_p]),
+    "nb_kl_vp_state": (c_int, [c_void_p, c_int64, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_float,
+                               c_float, c_void_p, c_void_p, c_size_t, c_void_p]),
+    "nb_kl_vp_combine": (c_int, [c_int64, c_int, c_void_p, c_void_p, c_int64, c_float, c_void_p, c_void_p,
+                                 c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p]),
+    "nb_kl_vp_jsd_partial": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_float,
+                                     c_float, c_void_p, c_void_p, c_void_p, c_void_p, c_size_t, c_void_p]),
+    "nb_kl_vp_jsd_combine": (c_int, [c_int64, c_int, c_void_p, c_void_p, c_int64, c_void_p, c_void_p, c_void_p,
+                                     c_void_p, c_void_p]),
     "nb_kl_backward": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_float, c_float,
                                c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_int, c_void_p,
                                c_size_t, c_void_p]),

@@ -6,7 +6,8 @@ section "工程落地": ``forward_kl`` / ``reverse_kl`` taking the student and t
 hidden states, both unembeddings and a temperature):
 
 * :func:`kl_forward` / :func:`kl_backward` — one call each of ``nb_kl_forward`` /
-  ``nb_kl_backward`` with caller-visible outputs;
+  ``nb_kl_backward`` with caller-visible outputs (``side=True``: ``nb_kl_forward_side``,
+  adding the student's per-token entropy and sampled-token log-probability);
 * :func:`generalized_jsd`, :func:`forward_kl`, :func:`reverse_kl` — autograd-enabled
   scalar losses (gradients reach ``h_s`` and ``W_s`` only; the teacher is frozen).
 """
@@ -71,8 +72,12 @@ def _workspace(nbytes: int, device, workspace: Optional[torch.Tensor]) -> torch.
 
 def kl_forward(h_s, W_s, h_t, W_t, labels, beta: float = 1.0, tau: float = 1.0, *,
                ignore_index: int = IGNORE_INDEX, chunk_v: int = 0, workspace: Optional[torch.Tensor] = None,
-               out: Optional[dict] = None) -> dict:
-    """Per-token loss, both tempered LSEs, aux, masked mean and N_v (device tensors)."""
+               out: Optional[dict] = None, side: bool = False) -> dict:
+    """Per-token loss, both tempered LSEs, aux, masked mean and N_v (device tensors).
+
+    With ``side``, also ``entropy_s`` (entropy of the tempered student softmax) and
+    ``logp_label`` (its log-probability of each row's label), fp32 [N], 0 on masked rows.
+    """
     _check_inputs(h_s, W_s, h_t, W_t, labels)
     dev = h_s.device
     N = labels.shape[0]
@@ -85,12 +90,21 @@ def kl_forward(h_s, W_s, h_t, W_t, labels, beta: float = 1.0, tau: float = 1.0, 
             "aux": torch.empty(N, **f32), "loss_mean": torch.empty((), **f32),
             "n_valid": torch.empty((), dtype=torch.int64, device=dev),
         }
-    code = _abi.lib().nb_kl_forward(
-        _abi.shape_ptr(shape), h_s.data_ptr(), W_s.data_ptr(), h_t.data_ptr(), W_t.data_ptr(), labels.data_ptr(),
-        float(beta), float(tau), out["loss_tok"].data_ptr(), out["lse_s"].data_ptr(), out["lse_t"].data_ptr(),
-        out["aux"].data_ptr(), out["loss_mean"].data_ptr(), out["n_valid"].data_ptr(), ws.data_ptr(),
-        ws.numel() * ws.element_size(), _stream_ptr(dev))
-    _abi.check("nb_kl_forward", code)
+        if side:
+            out["entropy_s"] = torch.empty(N, **f32)
+            out["logp_label"] = torch.empty(N, **f32)
+    common = (_abi.shape_ptr(shape), h_s.data_ptr(), W_s.data_ptr(), h_t.data_ptr(), W_t.data_ptr(),
+              labels.data_ptr(), float(beta), float(tau), out["loss_tok"].data_ptr(), out["lse_s"].data_ptr(),
+              out["lse_t"].data_ptr(), out["aux"].data_ptr(), out["loss_mean"].data_ptr(),
+              out["n_valid"].data_ptr())
+    tail = (ws.data_ptr(), ws.numel() * ws.element_size(), _stream_ptr(dev))
+    if side:
+        code = _abi.lib().nb_kl_forward_side(*common, out["entropy_s"].data_ptr(), out["logp_label"].data_ptr(),
+                                             *tail)
+        _abi.check("nb_kl_forward_side", code)
+    else:
+        code = _abi.lib().nb_kl_forward(*common, *tail)
+        _abi.check("nb_kl_forward", code)
     out["workspace"] = ws
     return out
 

@@ -80,13 +80,17 @@ struct SweepArgs {
   int tiles_per_unit;     // vocabulary tiles per work unit (one split of the LSE state)
   float scale;            // log2(e) / tau: base-2 tempered logits x = z * scale
   float beta, lg2_1mb, lg2_b;
-  float* out;             // state [5][split][ld] or JSD partial sums [2][split][ld]; split =
+  float* out;             // state [6][split][ld] or JSD partial sums [2][split][ld]; split =
                           // 2 * unit + column half
   long long field_stride; // elements between fields of `out`
   int ld;                 // rows per split in `out`
   const float* row_l2s;   // per compacted row: base-2 LSE of the student (pass 2, backward)
   const float* row_l2t;
   const float* row_aux;   // per compacted row: per-token KL (beta = 1) or KL(S||M) (JSD)
+  int side;               // forward state passes: also the student entropy accumulator and the
+                          // tempered logit of each row's label
+  const int* row_label;   // per compacted row: label column, or -1 (side outputs)
+  float* label_x;         // per compacted row: base-2 tempered student logit at the label
   __nv_bfloat16* G;       // backward: gradient chunk [rows][ldG]
   long long ldG;
   const float* gscale;    // device scalar grad_out / (N_v * tau)

@@ -66,8 +66,8 @@ struct Layout {
   int n_vt, n_split;
   int64_t chunk_v;
   int n_chunks;          // backward vocabulary chunks
-  size_t off_idx, off_hs, off_ht, off_rl2s, off_rl2t, off_raux, off_sched, off_dhc, off_state, off_part, off_G,
-      g_bytes, total;
+  size_t off_idx, off_hs, off_ht, off_rl2s, off_rl2t, off_raux, off_rlab, off_labx, off_sched, off_dhc, off_state,
+      off_part, off_G, g_bytes, total;
   long long fs_state;    // elements between state fields
 };
 
@@ -107,11 +107,13 @@ bool make_layout(const nb_kl_shape* sh, float beta, Layout& L) {
   L.off_rl2s = off;  off = align256(off + size_t(L.N_pad) * 4);
   L.off_rl2t = off;  off = align256(off + size_t(L.N_pad) * 4);
   L.off_raux = off;  off = align256(off + size_t(L.N_pad) * 4);
+  L.off_rlab = off;  off = align256(off + size_t(L.N_pad) * 4);   // label column per valid row
+  L.off_labx = off;  off = align256(off + size_t(L.N_pad) * 4);   // student logit at the label
   L.n_chunks = int((L.V + L.chunk_v - 1) / L.chunk_v);
   L.off_sched = off; off = align256(off + size_t(2 * L.n_chunks + 2) * 4);   // one work counter per launch
   L.off_dhc = off;   off = align256(off + size_t(L.N_pad) * L.d_s * 4);        // compacted dh_s (backward)
   // the forward's split state and the backward's two gradient-chunk buffers share one region
-  const size_t state_bytes = align256(size_t(5) * L.n_split * L.N_pad * 4);
+  const size_t state_bytes = align256(size_t(6) * L.n_split * L.N_pad * 4);
   const size_t part_bytes = jsd ? align256(size_t(2) * L.n_split * L.N_pad * 4) : 0;
   L.g_bytes = align256(size_t(L.N_pad) * L.chunk_v * 2);
   L.off_state = off;
@@ -278,6 +280,8 @@ struct Ws {
   float* dhc;
   __nv_bfloat16 *hs, *ht;
   float *rl2s, *rl2t, *raux, *state, *part;
+  int* rlab;
+  float* labx;
   __nv_bfloat16* G;
 };
 
@@ -293,6 +297,8 @@ Ws carve(const Layout& L, void* ws) {
   w.rl2s = reinterpret_cast<float*>(b + L.off_rl2s);
   w.rl2t = reinterpret_cast<float*>(b + L.off_rl2t);
   w.raux = reinterpret_cast<float*>(b + L.off_raux);
+  w.rlab = reinterpret_cast<int*>(b + L.off_rlab);
+  w.labx = reinterpret_cast<float*>(b + L.off_labx);
   w.state = reinterpret_cast<float*>(b + L.off_state);
   w.part = reinterpret_cast<float*>(b + L.off_part);
   w.G = reinterpret_cast<__nv_bfloat16*>(b + L.off_G);
@@ -410,6 +416,175 @@ nb_status fixed_scratch(void** out) {
   return NB_OK;
 }
 
+// Common start of the state-sweep forward calls: compaction of the valid rows (with the
+// label column of each row relative to the vocabulary range [v_off, v_off + V) when `side`),
+// bf16 gathers of both hidden states, the zeroed work counters and the sweep's tensor maps.
+struct Prep {
+  Layout L;
+  Ws w;
+  DevInfo dev;
+  cudaStream_t st;
+  SweepMaps maps;
+  SweepArgs a;
+};
+
+nb_status prepare(Prep& P, const nb_kl_shape* shape, const void* h_s, const void* W_s, const void* h_t,
+                  const void* W_t, const int64_t* labels, float beta, float tau, int side, int64_t v_off,
+                  int64_t* n_valid, void* workspace, cudaStream_t st) {
+  const Layout& L = P.L;
+  P.st = st;
+  P.w = carve(L, workspace);
+  const Ws& w = P.w;
+  // all-ones bits are a NaN: a label column the sweep never meets leaves a NaN log-probability
+  if (side && cudaMemsetAsync(w.labx, 0xFF, size_t(L.N_pad) * 4, st) != cudaSuccess) return NB_ERR_CUDA;
+  launch(compact_kernel, dim3(1), dim3(kScanThreads), 0, st, labels, int(L.N), (long long)shape->ignore_index,
+         w.idx, w.ctrl, n_valid, (const float*)nullptr, tau, side ? w.rlab : (int*)nullptr, (long long)L.V,
+         (long long)v_off);
+  launch_gather(L, w, h_s, L.d_s, w.hs, L.lda_s, st);
+  launch_gather(L, w, h_t, L.d_t, w.ht, L.lda_t, st);
+  if (cudaMemsetAsync(w.sched, 0, size_t(2 * L.n_chunks + 2) * 4, st) != cudaSuccess) return NB_ERR_CUDA;
+  if (!sweep_maps(L, w, W_s, W_t, P.maps)) return NB_ERR_CUDA;
+  P.a = base_sweep_args(L, w, beta, tau);
+  P.a.out = w.state;
+  P.a.sched = w.sched;
+  P.a.side = side;
+  P.a.row_label = w.rlab;
+  P.a.label_x = w.labx;
+  return NB_OK;
+}
+
+// The state sweep of the method's direction; returns the merge's kl_dir.
+int launch_state_sweep(const Prep& P, float beta) {
+  if (beta == 1.f) {
+    launch_sweep<kStateS>(P.dev, P.L, P.maps, P.a, P.st);
+    return 1;
+  }
+  if (beta == 0.f) {
+    launch_sweep<kStateT>(P.dev, P.L, P.maps, P.a, P.st);
+    return 2;
+  }
+  launch_sweep<kStateNone>(P.dev, P.L, P.maps, P.a, P.st);
+  return 0;
+}
+
+// Second JSD sweep (per-row base-2 LSEs already in row_l2s / row_l2t) and its reduction
+// into out_js / out_ks [N] in nats.
+void launch_jsd_pass(const Prep& P, float* out_js, float* out_ks) {
+  SweepArgs b = P.a;
+  b.side = 0;
+  b.out = P.w.part;
+  b.sched = P.w.sched + 1;
+  launch_sweep<kJsd>(P.dev, P.L, P.maps, b, P.st);
+  const unsigned rb = unsigned((P.L.N_pad + kMergeRows - 1) / kMergeRows);
+  launch(jsd_finalize_kernel, dim3(rb), dim3(kMergeRows * kMergeLanes), 0, P.st, (const float*)P.w.part,
+         (long long)P.L.fs_state, int(P.L.N_pad), P.L.n_split, (const int*)P.w.idx, (const Ctrl*)P.w.ctrl, out_js,
+         out_ks);
+}
+
+void launch_merge(const Prep& P, int kl_dir, int side, float* loss_tok, float* lse_s, float* lse_t, float* aux,
+                  float* entropy_s, float* logp_label, float* vp_state) {
+  const unsigned rb = unsigned((P.L.N_pad + kMergeRows - 1) / kMergeRows);
+  launch(merge_kernel, dim3(rb), dim3(kMergeRows * kMergeLanes), 0, P.st, (const float*)P.w.state,
+         (long long)P.L.fs_state, int(P.L.N_pad), P.L.n_split, (const int*)P.w.idx, (const Ctrl*)P.w.ctrl, kl_dir,
+         loss_tok, lse_s, lse_t, aux, P.w.rl2s, P.w.rl2t, side, (const float*)P.w.labx, entropy_s, logp_label,
+         vp_state, (long long)P.L.N);
+}
+
+nb_status zero_f32(float* p, int64_t n, cudaStream_t st) {
+  return (!p || cudaMemsetAsync(p, 0, size_t(n) * 4, st) == cudaSuccess) ? NB_OK : NB_ERR_CUDA;
+}
+
+// One forward call; with `entropy_s` / `logp_label` (either may be null) the state sweep also
+// produces the student's per-token side outputs.
+nb_status forward_impl(const nb_kl_shape* shape, const void* h_s, const void* W_s, const void* h_t, const void* W_t,
+                       const int64_t* labels, float beta, float tau, float* loss_tok, float* lse_s, float* lse_t,
+                       float* aux, float* loss_mean, int64_t* n_valid, float* entropy_s, float* logp_label,
+                       void* workspace, size_t workspace_bytes, void* stream) {
+  g_launches = 0;
+  Prep P;
+  nb_status s = validate_common(shape, h_s, W_s, h_t, W_t, labels, beta, tau, workspace, workspace_bytes, P.L);
+  if (s != NB_OK) return s;
+  const Layout& L = P.L;
+  if (!loss_mean || !n_valid) return NB_ERR_INVALID_ARG;
+  if (L.N > 0 && (!loss_tok || !lse_s || !lse_t || !aux)) return NB_ERR_INVALID_ARG;
+  const int side = (entropy_s || logp_label) ? 1 : 0;
+  if ((s = device_info(P.dev)) != NB_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(workspace, 0, kCtrlBytes, st) != cudaSuccess) return NB_ERR_CUDA;
+  if (L.N == 0) {
+    if (cudaMemsetAsync(loss_mean, 0, sizeof(float), st) != cudaSuccess) return NB_ERR_CUDA;
+    if (cudaMemsetAsync(n_valid, 0, sizeof(int64_t), st) != cudaSuccess) return NB_ERR_CUDA;
+    return NB_OK;
+  }
+  for (float* o : {loss_tok, lse_s, lse_t, aux, entropy_s, logp_label})
+    if ((s = zero_f32(o, L.N, st)) != NB_OK) return s;
+  if ((s = prepare(P, shape, h_s, W_s, h_t, W_t, labels, beta, tau, side, 0, n_valid, workspace, st)) !=
+      NB_OK)
+    return s;
+  const int kl_dir = launch_state_sweep(P, beta);
+  launch_merge(P, kl_dir, side, loss_tok, lse_s, lse_t, aux, entropy_s, logp_label, nullptr);
+  if (kl_dir == 0) launch_jsd_pass(P, loss_tok, aux);
+  launch(mean_kernel, dim3(1), dim3(1024), 0, st, (const float*)loss_tok, int(L.N), (const Ctrl*)P.w.ctrl,
+         loss_mean);
+  return check_launch();
+}
+
+// Vocabulary-parallel forward, first part: this rank's shard of the vocabulary (rows
+// [v_off, v_off + V) of the full unembeddings). Writes the shard's merged per-token state.
+nb_status vp_state_impl(const nb_kl_shape* shape, int64_t v_off, const void* h_s, const void* W_s, const void* h_t,
+                        const void* W_t, const int64_t* labels, float beta, float tau, float* state,
+                        void* workspace, size_t workspace_bytes, cudaStream_t st) {
+  g_launches = 0;
+  Prep P;
+  nb_status s = validate_common(shape, h_s, W_s, h_t, W_t, labels, beta, tau, workspace, workspace_bytes, P.L);
+  if (s != NB_OK) return s;
+  if (v_off < 0 || v_off > (int64_t(1) << 30)) return NB_ERR_INVALID_ARG;
+  if (P.L.N > 0 && !state) return NB_ERR_INVALID_ARG;
+  if ((s = device_info(P.dev)) != NB_OK) return s;
+  if (cudaMemsetAsync(workspace, 0, kCtrlBytes, st) != cudaSuccess) return NB_ERR_CUDA;
+  if (P.L.N == 0) return NB_OK;
+  if ((s = zero_f32(state, int64_t(kVpFields) * P.L.N, st)) != NB_OK) return s;
+  if ((s = prepare(P, shape, h_s, W_s, h_t, W_t, labels, beta, tau, 1, v_off, nullptr, workspace, st)) !=
+      NB_OK)
+    return s;
+  const int kl_dir = launch_state_sweep(P, beta);
+  launch_merge(P, kl_dir, 1, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, state);
+  return check_launch();
+}
+
+// Vocabulary-parallel JSD, second sweep over this rank's shard with the global LSEs:
+// per-token partial sums [2][N] in nats (the divergence and KL(S||M) over the shard).
+nb_status vp_jsd_partial_impl(const nb_kl_shape* shape, const void* h_s, const void* W_s, const void* h_t,
+                              const void* W_t, const int64_t* labels, float beta, float tau, const float* lse_s,
+                              const float* lse_t, float* part, void* workspace, size_t workspace_bytes,
+                              cudaStream_t st) {
+  g_launches = 0;
+  Prep P;
+  nb_status s = validate_common(shape, h_s, W_s, h_t, W_t, labels, beta, tau, workspace, workspace_bytes, P.L);
+  if (s != NB_OK) return s;
+  if (!(beta > 0.f && beta < 1.f)) return NB_ERR_INVALID_ARG;
+  if (P.L.N > 0 && (!lse_s || !lse_t || !part)) return NB_ERR_INVALID_ARG;
+  if ((s = device_info(P.dev)) != NB_OK) return s;
+  if (cudaMemsetAsync(workspace, 0, kCtrlBytes, st) != cudaSuccess) return NB_ERR_CUDA;
+  if (P.L.N == 0) return NB_OK;
+  if ((s = zero_f32(part, 2 * P.L.N, st)) != NB_OK) return s;
+  P.st = st;
+  P.w = carve(P.L, workspace);
+  const Layout& L = P.L;
+  const Ws& w = P.w;
+  launch(compact_kernel, dim3(1), dim3(kScanThreads), 0, st, labels, int(L.N), (long long)shape->ignore_index,
+         w.idx, w.ctrl, (int64_t*)nullptr, (const float*)nullptr, tau, (int*)nullptr, (long long)L.V, 0ll);
+  // the global LSEs become the per-row base-2 constants of the second pass (aux is unused there)
+  launch_gather(L, w, h_s, L.d_s, w.hs, L.lda_s, st, lse_s, lse_t, lse_s);
+  launch_gather(L, w, h_t, L.d_t, w.ht, L.lda_t, st);
+  if (cudaMemsetAsync(w.sched, 0, size_t(2 * L.n_chunks + 2) * 4, st) != cudaSuccess) return NB_ERR_CUDA;
+  if (!sweep_maps(L, w, W_s, W_t, P.maps)) return NB_ERR_CUDA;
+  P.a = base_sweep_args(L, w, beta, tau);
+  P.a.sched = w.sched;
+  launch_jsd_pass(P, part, part + L.N);
+  return check_launch();
+}
+
 }  // namespace
 
 // =====================================================================================
@@ -473,61 +648,74 @@ nb_status nb_kl_forward(const nb_kl_shape* shape, const void* h_s, const void* W
                         const void* W_t, const int64_t* labels, float beta, float tau, float* loss_tok,
                         float* lse_s, float* lse_t, float* aux, float* loss_mean, int64_t* n_valid,
                         void* workspace, size_t workspace_bytes, void* stream) {
+  return forward_impl(shape, h_s, W_s, h_t, W_t, labels, beta, tau, loss_tok, lse_s, lse_t, aux, loss_mean, n_valid,
+                      nullptr, nullptr, workspace, workspace_bytes, stream);
+}
+
+nb_status nb_kl_forward_side(const nb_kl_shape* shape, const void* h_s, const void* W_s, const void* h_t,
+                             const void* W_t, const int64_t* labels, float beta, float tau, float* loss_tok,
+                             float* lse_s, float* lse_t, float* aux, float* loss_mean, int64_t* n_valid,
+                             float* entropy_s, float* logp_label, void* workspace, size_t workspace_bytes,
+                             void* stream) {
+  return forward_impl(shape, h_s, W_s, h_t, W_t, labels, beta, tau, loss_tok, lse_s, lse_t, aux, loss_mean, n_valid,
+                      entropy_s, logp_label, workspace, workspace_bytes, stream);
+}
+
+nb_status nb_kl_vp_state(const nb_kl_shape* shape, int64_t vocab_offset, const void* h_s, const void* W_s,
+                         const void* h_t, const void* W_t, const int64_t* labels, float beta, float tau,
+                         float* state, void* workspace, size_t workspace_bytes, void* stream) {
+  return vp_state_impl(shape, vocab_offset, h_s, W_s, h_t, W_t, labels, beta, tau, state, workspace,
+                       workspace_bytes, static_cast<cudaStream_t>(stream));
+}
+
+nb_status nb_kl_vp_combine(int64_t n_tokens, int n_parts, const float* states, const int64_t* labels,
+                           int64_t ignore_index, float beta, float* loss_tok, float* lse_s, float* lse_t, float* aux,
+                           float* entropy_s, float* logp_label, float* loss_mean, int64_t* n_valid, void* stream) {
   g_launches = 0;
-  Layout L;
-  nb_status s = validate_common(shape, h_s, W_s, h_t, W_t, labels, beta, tau, workspace, workspace_bytes, L);
-  if (s != NB_OK) return s;
+  if (n_tokens < 0 || n_tokens > (int64_t(1) << 30) || n_parts < 1 || n_parts > 4096) return NB_ERR_INVALID_ARG;
+  if (!(beta >= 0.f && beta <= 1.f)) return NB_ERR_INVALID_ARG;
   if (!loss_mean || !n_valid) return NB_ERR_INVALID_ARG;
-  if (L.N > 0 && (!loss_tok || !lse_s || !lse_t || !aux)) return NB_ERR_INVALID_ARG;
-  DevInfo dev;
-  if ((s = device_info(dev)) != NB_OK) return s;
+  if (n_tokens > 0 && (!states || !labels || !loss_tok || !lse_s || !lse_t || !aux)) return NB_ERR_INVALID_ARG;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const Ws w = carve(L, workspace);
-  if (cudaMemsetAsync(w.ctrl, 0, kCtrlBytes, st) != cudaSuccess) return NB_ERR_CUDA;
-  if (L.N == 0) {
+  if (n_tokens == 0) {
     if (cudaMemsetAsync(loss_mean, 0, sizeof(float), st) != cudaSuccess) return NB_ERR_CUDA;
     if (cudaMemsetAsync(n_valid, 0, sizeof(int64_t), st) != cudaSuccess) return NB_ERR_CUDA;
     return NB_OK;
   }
-  const size_t nb = size_t(L.N) * sizeof(float);
-  if (cudaMemsetAsync(loss_tok, 0, nb, st) != cudaSuccess || cudaMemsetAsync(lse_s, 0, nb, st) != cudaSuccess ||
-      cudaMemsetAsync(lse_t, 0, nb, st) != cudaSuccess || cudaMemsetAsync(aux, 0, nb, st) != cudaSuccess)
-    return NB_ERR_CUDA;
+  const int kl_dir = beta == 1.f ? 1 : beta == 0.f ? 2 : 0;
+  launch(vp_combine_kernel, dim3(unsigned((n_tokens + 127) / 128)), dim3(128), 0, st, states, n_parts,
+         (long long)n_tokens, labels, (long long)ignore_index, kl_dir, loss_tok, lse_s, lse_t, aux, entropy_s,
+         logp_label);
+  launch(mean_count_kernel, dim3(1), dim3(1024), 0, st, (const float*)loss_tok, labels, (long long)n_tokens,
+         (long long)ignore_index, loss_mean, n_valid);
+  return check_launch();
+}
 
-  launch(compact_kernel, dim3(1), dim3(kScanThreads), 0, st, labels, int(L.N), (long long)shape->ignore_index,
-         w.idx, w.ctrl, n_valid, (const float*)nullptr, tau);
-  launch_gather(L, w, h_s, L.d_s, w.hs, L.lda_s, st);
-  launch_gather(L, w, h_t, L.d_t, w.ht, L.lda_t, st);
+nb_status nb_kl_vp_jsd_partial(const nb_kl_shape* shape, const void* h_s, const void* W_s, const void* h_t,
+                               const void* W_t, const int64_t* labels, float beta, float tau, const float* lse_s,
+                               const float* lse_t, float* part, void* workspace, size_t workspace_bytes,
+                               void* stream) {
+  return vp_jsd_partial_impl(shape, h_s, W_s, h_t, W_t, labels, beta, tau, lse_s, lse_t, part, workspace,
+                             workspace_bytes, static_cast<cudaStream_t>(stream));
+}
 
-  if (cudaMemsetAsync(w.sched, 0, size_t(2 * L.n_chunks + 2) * 4, st) != cudaSuccess) return NB_ERR_CUDA;
-  SweepMaps maps;
-  if (!sweep_maps(L, w, W_s, W_t, maps)) return NB_ERR_CUDA;
-  SweepArgs a = base_sweep_args(L, w, beta, tau);
-  a.out = w.state;
-  a.sched = w.sched;
-  int kl_dir = 0;
-  if (beta == 1.f) {
-    launch_sweep<kStateS>(dev, L, maps, a, st);
-    kl_dir = 1;
-  } else if (beta == 0.f) {
-    launch_sweep<kStateT>(dev, L, maps, a, st);
-    kl_dir = 2;
-  } else {
-    launch_sweep<kStateNone>(dev, L, maps, a, st);
+nb_status nb_kl_vp_jsd_combine(int64_t n_tokens, int n_parts, const float* parts, const int64_t* labels,
+                               int64_t ignore_index, float* loss_tok, float* aux, float* loss_mean, int64_t* n_valid,
+                               void* stream) {
+  g_launches = 0;
+  if (n_tokens < 0 || n_tokens > (int64_t(1) << 30) || n_parts < 1 || n_parts > 4096) return NB_ERR_INVALID_ARG;
+  if (!loss_mean || !n_valid) return NB_ERR_INVALID_ARG;
+  if (n_tokens > 0 && (!parts || !labels || !loss_tok || !aux)) return NB_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (n_tokens == 0) {
+    if (cudaMemsetAsync(loss_mean, 0, sizeof(float), st) != cudaSuccess) return NB_ERR_CUDA;
+    if (cudaMemsetAsync(n_valid, 0, sizeof(int64_t), st) != cudaSuccess) return NB_ERR_CUDA;
+    return NB_OK;
   }
-  const unsigned rb = unsigned((L.N_pad + kMergeRows - 1) / kMergeRows);
-  launch(merge_kernel, dim3(rb), dim3(kMergeRows * kMergeLanes), 0, st, (const float*)w.state, (long long)L.fs_state, int(L.N_pad),
-         L.n_split, (const int*)w.idx, (const Ctrl*)w.ctrl, kl_dir, loss_tok, lse_s, lse_t, aux, w.rl2s, w.rl2t);
-  if (kl_dir == 0) {
-    SweepArgs b = a;
-    b.out = w.part;
-    b.sched = w.sched + 1;
-    launch_sweep<kJsd>(dev, L, maps, b, st);
-    launch(jsd_finalize_kernel, dim3(rb), dim3(kMergeRows * kMergeLanes), 0, st, (const float*)w.part, (long long)L.fs_state,
-           int(L.N_pad), L.n_split, (const int*)w.idx, (const Ctrl*)w.ctrl, loss_tok, aux);
-  }
-  launch(mean_kernel, dim3(1), dim3(1024), 0, st, (const float*)loss_tok, int(L.N), (const Ctrl*)w.ctrl,
-         loss_mean);
+  launch(vp_jsd_combine_kernel, dim3(unsigned((n_tokens + 127) / 128)), dim3(128), 0, st, parts, n_parts,
+         (long long)n_tokens, labels, (long long)ignore_index, loss_tok, aux);
+  launch(mean_count_kernel, dim3(1), dim3(1024), 0, st, (const float*)loss_tok, labels, (long long)n_tokens,
+         (long long)ignore_index, loss_mean, n_valid);
   return check_launch();
 }
 
@@ -552,7 +740,7 @@ nb_status nb_kl_backward(const nb_kl_shape* shape, const void* h_s, const void* 
     return NB_OK;
   }
   launch(compact_kernel, dim3(1), dim3(kScanThreads), 0, st, labels, int(L.N), (long long)shape->ignore_index,
-         w.idx, w.ctrl, (int64_t*)nullptr, grad_out, tau);
+         w.idx, w.ctrl, (int64_t*)nullptr, grad_out, tau, (int*)nullptr, (long long)L.V, 0ll);
   launch_gather(L, w, h_s, L.d_s, w.hs, L.lda_s, st, lse_s, lse_t, aux);
   launch_gather(L, w, h_t, L.d_t, w.ht, L.lda_t, st);
   launch(zero_masked_rows_kernel, dim3(unsigned(L.N)), dim3(128), 0, st, labels, (long long)shape->ignore_index,

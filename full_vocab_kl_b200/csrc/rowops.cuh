@@ -17,13 +17,17 @@ struct Ctrl {          // first bytes of every workspace
 };
 
 // ------------------------------------------------------------------ compaction (one block)
-// Stable list of valid rows: idx[i] = position of the i-th label != ignore_index.
+// Stable list of valid rows: idx[i] = position of the i-th label != ignore_index. With
+// `row_label`, also the label of each valid row as a column of the vocabulary range
+// [v_off, v_off + V) held here (-1 outside it).
 constexpr int kScanThreads = 1024;
 
 __global__ void __launch_bounds__(kScanThreads) compact_kernel(const int64_t* __restrict__ labels, int N,
                                                                long long ignore_index, int* __restrict__ idx,
                                                                Ctrl* ctrl, int64_t* n_valid_out,
-                                                               const float* grad_out, float tau) {
+                                                               const float* grad_out, float tau,
+                                                               int* __restrict__ row_label, long long V,
+                                                               long long v_off) {
   __shared__ int warp_sums[32];
   __shared__ int s_total;
   const int per = (N + kScanThreads - 1) / kScanThreads;
@@ -53,8 +57,12 @@ __global__ void __launch_bounds__(kScanThreads) compact_kernel(const int64_t* __
   }
   __syncthreads();
   int pos = warp_sums[warp] + incl - cnt;
-  for (int i = b; i < e; ++i)
-    if (labels[i] != ignore_index) idx[pos++] = i;
+  for (int i = b; i < e; ++i) {
+    const long long y = labels[i];
+    if (y == ignore_index) continue;
+    if (row_label) row_label[pos] = (y >= v_off && y - v_off < V) ? int(y - v_off) : -1;
+    idx[pos++] = i;
+  }
   if (threadIdx.x == 0) {
     const int nv = s_total;
     ctrl->n_valid = nv;
@@ -112,6 +120,9 @@ __global__ void gather_rows_kernel(const void* __restrict__ src, int d, __nv_bfl
 //   LSE(u) = ln 2 * (m + log2 l),  KL = ln 2 * (a / l_p - L2_p + L2_q)
 // `kl_dir`: 1 reverse (p = student), 2 forward (p = teacher), 0 none (JSD pass 1: the
 // base-2 LSEs go to row_l2s / row_l2t for the second pass).
+// With `side`, the student's entropy and label log-probability are written as well:
+//   H = ln 2 * (log2 l_s - E / l_s), E = sum_k 2^(m_k - M) (e_k + (m_k - M) l_k)
+//   log S[label] = ln 2 * (x_label - L2_s)  (NaN when the sweep saw no label column)
 // Block = 32 rows x 8 split lanes: lane j of row r visits splits j, j + 8, ... so that a warp
 // (32 consecutive rows, one split) reads contiguous memory; the 8 partial results of a row
 // are combined in shared memory in a fixed order.
@@ -120,9 +131,11 @@ constexpr int kMergeRows = 32, kMergeLanes = 8;
 __global__ void __launch_bounds__(kMergeRows * kMergeLanes)
     merge_kernel(const float* __restrict__ state, long long fs, int ld, int n_split, const int* __restrict__ idx,
                  const Ctrl* __restrict__ ctrl, int kl_dir, float* loss_tok, float* lse_s, float* lse_t, float* aux,
-                 float* row_l2s, float* row_l2t) {
+                 float* row_l2s, float* row_l2t, int side, const float* __restrict__ label_x, float* entropy_s,
+                 float* logp_label, float* vp_state, long long vp_ld) {
   __shared__ float sm_s[kMergeLanes][kMergeRows], sm_t[kMergeLanes][kMergeRows];
   __shared__ double sl_s[kMergeLanes][kMergeRows], sl_t[kMergeLanes][kMergeRows], sa[kMergeLanes][kMergeRows];
+  __shared__ double se[kMergeLanes][kMergeRows];
   const int r = threadIdx.x % kMergeRows, j = threadIdx.x / kMergeRows;
   const int nv = ctrl->n_valid;
   const int i = blockIdx.x * kMergeRows + r;
@@ -142,7 +155,7 @@ __global__ void __launch_bounds__(kMergeRows * kMergeLanes)
     ms = fmaxf(ms, sm_s[q][r]);
     mt = fmaxf(mt, sm_t[q][r]);
   }
-  double ls = 0.0, lt = 0.0, a = 0.0;
+  double ls = 0.0, lt = 0.0, a = 0.0, e = 0.0;
   if (live)
     for (int k = j; k < n_split; k += kMergeLanes) {
       const long long o = (long long)k * ld + i;
@@ -152,22 +165,39 @@ __global__ void __launch_bounds__(kMergeRows * kMergeLanes)
       lt += state[3 * fs + o] * ft_;
       if (kl_dir == 1) a += state[4 * fs + o] * fs_;
       if (kl_dir == 2) a += state[4 * fs + o] * ft_;
+      if (side) e += (double(state[5 * fs + o]) + (double(state[o]) - ms) * state[fs + o]) * fs_;
     }
   sl_s[j][r] = ls;
   sl_t[j][r] = lt;
   sa[j][r] = a;
+  se[j][r] = e;
   __syncthreads();
   if (j != 0 || !live) return;
-  ls = lt = a = 0.0;
+  ls = lt = a = e = 0.0;
   for (int q = 0; q < kMergeLanes; ++q) {
     ls += sl_s[q][r];
     lt += sl_t[q][r];
     a += sa[q][r];
+    e += se[q][r];
+  }
+  const int row = idx[i];
+  if (vp_state) {   // one vocabulary shard: its merged state, finished by vp_combine_kernel
+    vp_state[row] = ms;
+    vp_state[vp_ld + row] = float(ls);
+    vp_state[2 * vp_ld + row] = mt;
+    vp_state[3 * vp_ld + row] = float(lt);
+    vp_state[4 * vp_ld + row] = float(a);
+    vp_state[5 * vp_ld + row] = float(e);
+    vp_state[6 * vp_ld + row] = side ? label_x[i] : __int_as_float(0x7fffffff);
+    return;
   }
   const double L2s = ms + log2(ls), L2t = mt + log2(lt);
-  const int row = idx[i];
   lse_s[row] = float(L2s * 0.69314718055994530942);
   lse_t[row] = float(L2t * 0.69314718055994530942);
+  if (side) {
+    if (entropy_s) entropy_s[row] = float(0.69314718055994530942 * (log2(ls) - e / ls));
+    if (logp_label) logp_label[row] = float(0.69314718055994530942 * (double(label_x[i]) - L2s));
+  }
   if (kl_dir == 1) {
     const float kl = float(0.69314718055994530942 * (a / ls - L2s + L2t));
     loss_tok[row] = kl;
@@ -209,6 +239,108 @@ __global__ void __launch_bounds__(kMergeRows * kMergeLanes)
   const int row = idx[i];
   loss_tok[row] = float(js * 0.69314718055994530942);
   aux[row] = float(ks * 0.69314718055994530942);
+}
+
+// ------------------------------------------------------------------ vocabulary-parallel combine
+// Exchange format of one vocabulary shard, field-major [kVpFields][n_tokens] fp32, base-2
+// tempered units (x = u log2 e): m_s, l_s, m_t, l_t, a, e (see merge_kernel) and the student
+// logit at the row's label (NaN when the label is not in the shard).
+constexpr int kVpFields = 7;
+
+// Merge the states of `n_parts` shards ([part][field][n_tokens], fixed part order, fp64
+// sums) and finish each valid row exactly as merge_kernel does for one GPU; masked rows get
+// 0 everywhere. kl_dir 0 (JSD) writes the LSEs and side outputs only (loss and aux come
+// from the second pass).
+__global__ void __launch_bounds__(128)
+    vp_combine_kernel(const float* __restrict__ st, int n_parts, long long N, const int64_t* __restrict__ labels,
+                      long long ignore_index, int kl_dir, float* loss_tok, float* lse_s, float* lse_t, float* aux,
+                      float* entropy_s, float* logp_label) {
+  const long long row = blockIdx.x * 128ll + threadIdx.x;
+  if (row >= N) return;
+  const long long P = (long long)kVpFields * N;   // elements per part
+  if (labels[row] == ignore_index) {
+    loss_tok[row] = 0.f;
+    lse_s[row] = 0.f;
+    lse_t[row] = 0.f;
+    aux[row] = 0.f;
+    if (entropy_s) entropy_s[row] = 0.f;
+    if (logp_label) logp_label[row] = 0.f;
+    return;
+  }
+  float ms = kNegBig, mt = kNegBig;
+  for (int k = 0; k < n_parts; ++k) {
+    ms = fmaxf(ms, st[k * P + row]);
+    mt = fmaxf(mt, st[k * P + 2 * N + row]);
+  }
+  double ls = 0.0, lt = 0.0, a = 0.0, e = 0.0;
+  float xl = __int_as_float(0x7fffffff);
+  for (int k = 0; k < n_parts; ++k) {
+    const float* q = st + k * P;
+    const double fs_ = exp2(double(q[row]) - ms), ft_ = exp2(double(q[2 * N + row]) - mt);
+    ls += q[N + row] * fs_;
+    lt += q[3 * N + row] * ft_;
+    if (kl_dir == 1) a += q[4 * N + row] * fs_;
+    if (kl_dir == 2) a += q[4 * N + row] * ft_;
+    e += (double(q[5 * N + row]) + (double(q[row]) - ms) * q[N + row]) * fs_;
+    const float x = q[6 * N + row];
+    if (x == x && xl != xl) xl = x;   // first shard that holds the label
+  }
+  const double L2s = ms + log2(ls), L2t = mt + log2(lt);
+  lse_s[row] = float(L2s * 0.69314718055994530942);
+  lse_t[row] = float(L2t * 0.69314718055994530942);
+  if (entropy_s) entropy_s[row] = float(0.69314718055994530942 * (log2(ls) - e / ls));
+  if (logp_label) logp_label[row] = float(0.69314718055994530942 * (double(xl) - L2s));
+  float kl = 0.f;
+  if (kl_dir == 1) kl = float(0.69314718055994530942 * (a / ls - L2s + L2t));
+  if (kl_dir == 2) kl = float(0.69314718055994530942 * (a / lt - L2t + L2s));
+  loss_tok[row] = kl;
+  aux[row] = kl;
+}
+
+// JSD second pass across shards: per valid row, the fixed-order sum of the shards'
+// partial sums ([part][2][n_tokens], nats: the divergence and KL(S||M)).
+__global__ void __launch_bounds__(128)
+    vp_jsd_combine_kernel(const float* __restrict__ parts, int n_parts, long long N,
+                          const int64_t* __restrict__ labels, long long ignore_index, float* loss_tok, float* aux) {
+  const long long row = blockIdx.x * 128ll + threadIdx.x;
+  if (row >= N) return;
+  double js = 0.0, ks = 0.0;
+  if (labels[row] != ignore_index)
+    for (int k = 0; k < n_parts; ++k) {
+      js += parts[k * 2 * N + row];
+      ks += parts[k * 2 * N + N + row];
+    }
+  loss_tok[row] = float(js);
+  aux[row] = float(ks);
+}
+
+// Masked mean without a workspace: one block counts the valid labels and sums loss_tok
+// (masked rows hold 0) in a fixed order, in fp64.
+__global__ void __launch_bounds__(1024)
+    mean_count_kernel(const float* __restrict__ loss_tok, const int64_t* __restrict__ labels, long long N,
+                      long long ignore_index, float* loss_mean, int64_t* n_valid) {
+  __shared__ double part[1024];
+  __shared__ long long cnt[1024];
+  double s = 0.0;
+  long long c = 0;
+  for (long long i = threadIdx.x; i < N; i += 1024) {
+    s += loss_tok[i];
+    c += labels[i] != ignore_index;
+  }
+  part[threadIdx.x] = s;
+  cnt[threadIdx.x] = c;
+  __syncthreads();
+  for (int o = 512; o > 0; o >>= 1) {
+    if (threadIdx.x < o) {
+      part[threadIdx.x] += part[threadIdx.x + o];
+      cnt[threadIdx.x] += cnt[threadIdx.x + o];
+    }
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) {
+    *loss_mean = cnt[0] > 0 ? float(part[0] / double(cnt[0])) : 0.f;
+    if (n_valid) *n_valid = cnt[0];
+  }
 }
 
 // Deterministic masked mean: fixed-order fp64 sum of loss_tok (masked rows hold 0).

@@ -293,12 +293,15 @@ __device__ __forceinline__ void sweep_mma(const SweepArgs& p, const UnitGrid& g,
 // ------------------------------------------------------------------ epilogue math
 // Online base-2 state of one token row: running maxima m, rescaled sums l = sum 2^(x - m),
 // and a = sum 2^(x_p - m_p) (x_p - x_q) for the model p the KL takes its expectation under.
+// With side outputs, e = sum 2^(x_s - m_s) (x_s - m_s): every term is <= 0, so the student
+// entropy ln 2 * (log2 l_s - e / l_s) is formed without cancellation.
 struct RowState {
-  float ms, ls, mt, lt, a;
+  float ms, ls, mt, lt, a, e;
 };
 
-template <int MODE, bool MASKED>
-__device__ __forceinline__ void chunk_state(float (&zs)[32], float (&zt)[32], int n_ok, float scale, RowState& r) {
+template <int MODE, bool MASKED, bool SIDE>
+__device__ __forceinline__ void chunk_state(float (&zs)[32], float (&zt)[32], int n_ok, float scale, RowState& r,
+                                            int lab_off, float* lab_dst) {
   float cs = kNegBig, ct = kNegBig;
 #pragma unroll
   for (int j = 0; j < 32; ++j) {
@@ -311,25 +314,39 @@ __device__ __forceinline__ void chunk_state(float (&zs)[32], float (&zt)[32], in
   }
   const float ns = fmaxf(r.ms, cs), nt = fmaxf(r.mt, ct);
   const float rs = ex2(r.ms - ns), rt = ex2(r.mt - nt);
+  // re-centre e on the new maximum: sum 2^(x - ns) (x - ns) = rs (e + (ms - ns) l)
+  if (SIDE) r.e = rs * fmaf(r.ms - ns, r.ls, r.e);
   r.ls *= rs;
   r.lt *= rt;
   if (MODE == kStateS) r.a *= rs;
   if (MODE == kStateT) r.a *= rt;
   r.ms = ns;
   r.mt = nt;
-  float ls = 0.f, lt = 0.f, a = 0.f;
+  float ls = 0.f, lt = 0.f, a = 0.f, e = 0.f;
 #pragma unroll
   for (int j = 0; j < 32; ++j) {
-    const float es = ex2(zs[j] - ns);
+    const float ds = zs[j] - ns;
+    const float es = ex2(ds);
     const float et = ex2(zt[j] - nt);
     ls += es;
     lt += et;
+    if (SIDE) e = fmaf(es, ds, e);
     if (MODE == kStateS) a = fmaf(es, zs[j] - zt[j], a);
     if (MODE == kStateT) a = fmaf(et, zt[j] - zs[j], a);
   }
   r.ls += ls;
   r.lt += lt;
   r.a += a;
+  if (SIDE) {
+    r.e += e;
+    // the one thread whose chunk holds the row's label keeps that logit (a rare branch)
+    if (unsigned(lab_off) < 32u) {
+      float x = 0.f;
+#pragma unroll
+      for (int j = 0; j < 32; ++j) x = (j == lab_off) ? zs[j] : x;
+      *lab_dst = x;
+    }
+  }
 }
 
 struct RowConst {
@@ -400,11 +417,16 @@ __device__ __forceinline__ void chunk_grad(const float (&zs)[32], const float (&
 template <int MODE>
 __device__ __forceinline__ void process_chunk(float (&zs)[32], float (&zt)[32], int n_ok, const SweepArgs& p,
                                               const RowConst& c, float gs, RowState& r, float& js, float& ks,
-                                              uint8_t* gstage, int lane) {
+                                              uint8_t* gstage, int lane, int lab_off, float* lab_dst) {
   const bool masked = n_ok < 32;
   if (MODE <= kStateT) {
-    if (masked) chunk_state<MODE, true>(zs, zt, n_ok, p.scale, r);
-    else chunk_state<MODE, false>(zs, zt, n_ok, p.scale, r);
+    if (p.side) {
+      if (masked) chunk_state<MODE, true, true>(zs, zt, n_ok, p.scale, r, lab_off, lab_dst);
+      else chunk_state<MODE, false, true>(zs, zt, n_ok, p.scale, r, lab_off, lab_dst);
+    } else {
+      if (masked) chunk_state<MODE, true, false>(zs, zt, n_ok, p.scale, r, -1, nullptr);
+      else chunk_state<MODE, false, false>(zs, zt, n_ok, p.scale, r, -1, nullptr);
+    }
   } else if (MODE == kJsd) {
     if (masked) chunk_jsd<true>(zs, zt, n_ok, p.scale, c, js, ks);
     else chunk_jsd<false>(zs, zt, n_ok, p.scale, c, js, ks);
@@ -450,7 +472,10 @@ __device__ __forceinline__ void sweep_epilogue(const SweepMaps& maps, const Swee
       c.aux = p.row_aux[row];
     }
     const float gs = row_ok ? gscale : 0.f;
-    RowState r{kNegBig, 0.f, kNegBig, 0.f, 0.f};
+    // label column of this row (side outputs of the state passes), -1 when none
+    const int lab = (MODE <= kStateT && p.side && row_ok) ? p.row_label[row] : -1;
+    float* const lab_dst = (MODE <= kStateT && p.side) ? p.label_x + row : nullptr;
+    RowState r{kNegBig, 0.f, kNegBig, 0.f, 0.f, 0.f};
     float js = 0.f, ks = 0.f;
     const int t_end = min((vu + 1) * p.tiles_per_unit, g.n_vt);
     for (int t = vu * p.tiles_per_unit; t < t_end; ++t, ++lt) {
@@ -476,8 +501,9 @@ __device__ __forceinline__ void sweep_epilogue(const SweepMaps& maps, const Swee
           if (staged && lane == 0) bulk_wait_read();
           __syncwarp();
         }
-        if (p.teacher_first) process_chunk<MODE>(C, F[ch], n_ok, p, c, gs, r, js, ks, stage_row, lane);
-        else process_chunk<MODE>(F[ch], C, n_ok, p, c, gs, r, js, ks, stage_row, lane);
+        const int lab_off = lab < 0 ? -1 : lab - c0;
+        if (p.teacher_first) process_chunk<MODE>(C, F[ch], n_ok, p, c, gs, r, js, ks, stage_row, lane, lab_off, lab_dst);
+        else process_chunk<MODE>(F[ch], C, n_ok, p, c, gs, r, js, ks, stage_row, lane, lab_off, lab_dst);
         if (MODE >= kGradFkl) {
           fence_async_smem();
           __syncwarp();
@@ -496,6 +522,7 @@ __device__ __forceinline__ void sweep_epilogue(const SweepMaps& maps, const Swee
       p.out[2 * p.field_stride + off] = r.mt;
       p.out[3 * p.field_stride + off] = r.lt;
       p.out[4 * p.field_stride + off] = r.a;
+      if (p.side) p.out[5 * p.field_stride + off] = r.e;
     } else if (MODE == kJsd) {
       p.out[off] = js;
       p.out[p.field_stride + off] = ks;

@@ -87,6 +87,77 @@ NB_KL_API nb_status nb_kl_forward(const nb_kl_shape* shape, const void* h_s, con
                         float* lse_s, float* lse_t, float* aux, float* loss_mean, int64_t* n_valid,
                         void* workspace, size_t workspace_bytes, void* stream);
 
+/* Forward plus per-token side outputs of the student from the same sweep
+ * ("01 · 论文精读与参考实现全景映射", section 1: Eq. 6, the per-token entropy H_t that the
+ * peak-entropy scheduler of section 3.5 ranks; Eq. 8, log pi_theta(y_t | .) of the
+ * student's own sampled token). Both are taken under the tempered student softmax
+ * S = softmax(z_s / tau) that the loss uses, in nats:
+ *   entropy_s[n]  = -sum_v S[n,v] ln S[n,v]
+ *   logp_label[n] = ln S[n, labels[n]]   (NaN when labels[n] is outside [0, vocab))
+ * entropy_s and logp_label are device fp32 [n_tokens], caller-owned; either may be NULL
+ * (both NULL is nb_kl_forward). Masked rows get 0 in both. Every other argument and result
+ * is that of nb_kl_forward, with the same workspace. */
+NB_KL_API nb_status nb_kl_forward_side(const nb_kl_shape* shape, const void* h_s, const void* W_s,
+                             const void* h_t, const void* W_t, const int64_t* labels, float beta, float tau,
+                             float* loss_tok, float* lse_s, float* lse_t, float* aux, float* loss_mean,
+                             int64_t* n_valid, float* entropy_s, float* logp_label, void* workspace,
+                             size_t workspace_bytes, void* stream);
+
+/* ---- Vocabulary-parallel forward (the unembeddings split by rows across ranks) ----------
+ * "Nitrobrew tweet analysis", section "工程落地": under tensor parallelism the unembedding is
+ * sharded, and the full-vocabulary loss then needs one exchange per token. Each rank holds
+ * rows [vocab_offset, vocab_offset + shape->vocab) of W_s and W_t (W_s / W_t point at the
+ * shard) and the full h_s, h_t and labels. The per-token online softmax state of a shard is
+ * merged across shards with the same log-sum-exp merge the single-GPU call uses between its
+ * vocabulary splits, so the result equals the unsharded call up to summation order.
+ *
+ * Flow on every rank (the exchange is the caller's, e.g. an all-gather over NCCL):
+ *   nb_kl_vp_state      -> state  [NB_KL_VP_FIELDS][n_tokens]      (local shard)
+ *   all-gather          -> states [n_parts][NB_KL_VP_FIELDS][n_tokens] (parts in rank order)
+ *   nb_kl_vp_combine    -> lse_s, lse_t, entropy_s, logp_label; for beta in {0, 1} also
+ *                          loss_tok, aux, loss_mean, n_valid (final)
+ *   for 0 < beta < 1:  nb_kl_vp_jsd_partial (local shard, global lse_s / lse_t)
+ *                      -> part [2][n_tokens];  all-gather -> parts [n_parts][2][n_tokens];
+ *                      nb_kl_vp_jsd_combine -> loss_tok, aux, loss_mean, n_valid
+ * The backward needs no new call: nb_kl_backward on the shard with the global lse_s, lse_t
+ * and aux gives this shard's rows of dW_s exactly and its term of dh_s; dh_s is the sum of
+ * the ranks' terms (an all-reduce).
+ *
+ * State layout: fp32, field-major, base-2 tempered units (x = z log2(e) / tau): the running
+ * maxima and rescaled sums of both models (m_s, l_s, m_t, l_t), the KL numerator a (beta in
+ * {0, 1}), the student entropy accumulator e, and the student's x at the row's label (NaN
+ * when the label is not in this shard). Masked rows hold 0 and are never read. */
+#define NB_KL_VP_FIELDS 7
+
+/* First part on one shard. shape->vocab is the shard's row count; the workspace is sized by
+ * nb_kl_workspace_size(shape, beta). Labels keep their global values. */
+NB_KL_API nb_status nb_kl_vp_state(const nb_kl_shape* shape, int64_t vocab_offset, const void* h_s,
+                         const void* W_s, const void* h_t, const void* W_t, const int64_t* labels, float beta,
+                         float tau, float* state, void* workspace, size_t workspace_bytes, void* stream);
+
+/* Merge of n_parts gathered shard states (device, [n_parts][NB_KL_VP_FIELDS][n_tokens]) in
+ * part order, in fp64. Outputs as nb_kl_forward_side (entropy_s / logp_label may be NULL);
+ * for 0 < beta < 1, loss_tok and aux are written as 0 and loss_mean / n_valid are those of
+ * the zero losses: nb_kl_vp_jsd_combine replaces them. No workspace. */
+NB_KL_API nb_status nb_kl_vp_combine(int64_t n_tokens, int n_parts, const float* states, const int64_t* labels,
+                           int64_t ignore_index, float beta, float* loss_tok, float* lse_s, float* lse_t,
+                           float* aux, float* entropy_s, float* logp_label, float* loss_mean, int64_t* n_valid,
+                           void* stream);
+
+/* Second JSD sweep on one shard (0 < beta < 1 only) with the merged natural-log lse_s /
+ * lse_t [n_tokens]: part[0][n] = the shard's terms of the divergence of row n, part[1][n] =
+ * its terms of KL(S || M), in nats (device fp32 [2][n_tokens]; masked rows 0). */
+NB_KL_API nb_status nb_kl_vp_jsd_partial(const nb_kl_shape* shape, const void* h_s, const void* W_s,
+                               const void* h_t, const void* W_t, const int64_t* labels, float beta, float tau,
+                               const float* lse_s, const float* lse_t, float* part, void* workspace,
+                               size_t workspace_bytes, void* stream);
+
+/* Sum of n_parts gathered JSD partials ([n_parts][2][n_tokens]) in part order, in fp64:
+ * loss_tok, aux [n_tokens], loss_mean, n_valid. No workspace. */
+NB_KL_API nb_status nb_kl_vp_jsd_combine(int64_t n_tokens, int n_parts, const float* parts,
+                               const int64_t* labels, int64_t ignore_index, float* loss_tok, float* aux,
+                               float* loss_mean, int64_t* n_valid, void* stream);
+
 /* Backward ("仓库实现": recompute the logit blocks; gradients reach h_s and W_s only).
  * Inputs lse_s, lse_t, aux are the forward's outputs for the same arguments; grad_out is
  * one fp32 on the device (dOut/dloss_mean). Writes dh_s [n_tokens, d_s] (masked rows 0)

@@ -6,6 +6,10 @@ Tolerances (valid rows only):
   per-token loss  |d| <= 2e-3 |ref| + 1e-5 nats
   lse_s, lse_t    relative error <= 1e-5
   dh_s, dW_s      relative L2 error <= 1e-2
+Side outputs (valid rows only):
+  entropy_s       |d| <= 2e-3 |ref| + 1e-5 nats (the per-token loss bound)
+  logp_label      |d| <= 1e-5 (|lse_s| + |u_label|) + 1e-5 nats (the LSE bound carried
+                  through log S[y] = u_y - lse_s); NaN exactly where the label is outside [0, V)
 """
 
 import numpy as np
@@ -85,6 +89,25 @@ def check_forward(got, ref, labels, rows=None):
             assert got["loss_mean"] == 0.0
         else:
             assert abs(got["loss_mean"] - m) <= TOL_MEAN * abs(m) + 1e-7, (got["loss_mean"], m)
+
+
+def check_side(got, ref, labels, V, rows=None):
+    valid = labels != -100
+    sel = np.flatnonzero(valid) if rows is None else np.asarray([r for r in rows if valid[r]])
+    H, Hr = got["entropy_s"][sel], ref["entropy_s"][sel]
+    bad = ~(np.abs(H - Hr) <= TOL_TOK_REL * np.abs(Hr) + TOL_TOK_ABS)
+    assert not bad.any(), f"entropy: {bad.sum()} rows off, worst {np.abs(H - Hr)[bad].max()}"
+    lp, lpr = got["logp_label"][sel], ref["logp_label"][sel]
+    inside = (labels[sel] >= 0) & (labels[sel] < V)
+    assert np.isnan(lp[~inside]).all() and np.isnan(lpr[~inside]).all()
+    lp, lpr = lp[inside], lpr[inside]
+    lse = ref["lse_s"][sel][inside]
+    bound = TOL_LSE * (np.abs(lse) + np.abs(lpr + lse)) + 1e-5
+    bad = ~(np.abs(lp - lpr) <= bound)
+    assert not bad.any(), f"logp_label: {bad.sum()} rows off, worst {np.abs(lp - lpr)[bad].max()}"
+    masked = np.flatnonzero(~valid)
+    for k in ("entropy_s", "logp_label"):
+        assert (got[k][masked] == 0).all(), f"{k} not zero on masked rows"
 
 
 def oracle_all(x, beta=None, tau=None, labels=None, dW_init=None):

@@ -130,3 +130,26 @@ def test_python_api_refuses_cpu_tensors(L):
     x = torch.zeros(4, 8, dtype=torch.bfloat16)
     with pytest.raises(ValueError):
         nb.kl_forward(x, x, x, x, torch.zeros(4, dtype=torch.int64))
+
+
+def test_vocab_parallel_argument_errors(L):
+    lib = L.lib()
+    s = shape(L, N=256, V=1024, ds=256, dt=256)
+    p = [ctypes.c_void_p(v) for v in FAKE]
+    wsb = ws_size(L, s)
+    # negative shard offset
+    assert lib.nb_kl_vp_state(L.shape_ptr(s), -256, p[0], p[1], p[2], p[3], p[4], 1.0, 1.0, p[5], p[6], wsb,
+                              None) == L.NB_ERR_INVALID_ARG
+    # missing state output
+    assert lib.nb_kl_vp_state(L.shape_ptr(s), 0, p[0], p[1], p[2], p[3], p[4], 1.0, 1.0, None, p[6], wsb,
+                              None) == L.NB_ERR_INVALID_ARG
+    # no parts / bad beta
+    assert lib.nb_kl_vp_combine(256, 0, p[0], p[1], -100, 1.0, p[2], p[3], p[4], p[5], None, None, p[6], p[7],
+                                None) == L.NB_ERR_INVALID_ARG
+    assert lib.nb_kl_vp_combine(256, 2, p[0], p[1], -100, 2.0, p[2], p[3], p[4], p[5], None, None, p[6], p[7],
+                                None) == L.NB_ERR_INVALID_ARG
+    # the second JSD pass only exists for 0 < beta < 1
+    assert lib.nb_kl_vp_jsd_partial(L.shape_ptr(s), p[0], p[1], p[2], p[3], p[4], 1.0, 1.0, p[5], p[6], p[7],
+                                    p[8], wsb, None) == L.NB_ERR_INVALID_ARG
+    assert lib.nb_kl_vp_jsd_combine(256, 2, None, p[1], -100, p[2], p[3], p[4], p[5],
+                                    None) == L.NB_ERR_INVALID_ARG
