@@ -13,3 +13,4 @@ from .kl_oracle import (  # noqa: F401
     log_softmax,
     tempered_logits,
 )
+from . import spectral  # noqa: F401

@@ -145,3 +145,44 @@ def test_untempered_side_outputs_caught(monkeypatch):
     # at tau = 2: logS * 2 re-normalised is the softmax of z itself
     _side_mutant(monkeypatch, lambda o, lS, lab: o(ko.log_softmax(lS * 2.0)[0], lab))
     assert _fails(side_pins.test_two_level_closed_form, 3, 2.0, -1.0, 2.0)
+
+
+# ------------------------------------------------------------------ spectral front end
+import oracle.spectral as spo  # noqa: E402
+import test_oracle_spectral_pins as spec_pins  # noqa: E402
+
+
+def test_smallest_singular_vectors_caught(monkeypatch):
+    def bad(W, k):
+        W = np.asarray(W, dtype=np.float64)
+        _, s, vt = np.linalg.svd(W, full_matrices=False)
+        return vt[-k:][::-1].T.copy(), s[-k:][::-1].copy()
+    monkeypatch.setattr(spo, "spectral_basis", bad)
+    assert _fails(spec_pins.test_top_subspace_and_eckart_young)
+
+
+def test_transposed_singular_factor_caught(monkeypatch):
+    # columns of V^T taken where the rows were meant (a transposition slip)
+    def bad(W, k):
+        W = np.asarray(W, dtype=np.float64)
+        _, s, vt = np.linalg.svd(W, full_matrices=False)
+        return vt[:, :k].copy(), s[:k].copy()
+    monkeypatch.setattr(spo, "spectral_basis", bad)
+    assert _fails(spec_pins.test_top_subspace_and_eckart_young)
+
+
+def test_truncated_coordinates_instead_of_projection_caught(monkeypatch):
+    # keeping the first k coordinates of h instead of its coordinates in the basis
+    monkeypatch.setattr(spo, "project", lambda x, Vk: np.asarray(x, dtype=np.float64)[:, :Vk.shape[1]])
+    assert _fails(spec_pins.test_full_rank_and_exact_low_rank_are_lossless)
+
+
+def test_unscaled_teacher_unembedding_caught(monkeypatch):
+    # W_t' = U_k instead of U_k S_k: drop the singular values
+    orig = spo.compress_teacher
+
+    def bad(h, W, k):
+        hp, Wp, Vk = orig(h, W, k)
+        return hp, Wp / np.linalg.norm(Wp, axis=0, keepdims=True), Vk
+    monkeypatch.setattr(spo, "compress_teacher", bad)
+    assert _fails(spec_pins.test_closed_form_diagonal)
