@@ -23,6 +23,7 @@ NB_BF16 = 0
 NB_F32 = 1
 NOALLOC_SCRATCH_BYTES = 64 * 1024 * 1024
 VP_FIELDS = 7   # NB_KL_VP_FIELDS: floats per token of a vocabulary shard's state
+SMALL_WORKSPACE_BYTES = 256   # NB_KL_SMALL_WORKSPACE_BYTES
 
 # every function the header declares, with (restype, argtypes)
 SIGNATURES = {
@@ -41,6 +42,8 @@ SIGNATURES = {
                                      c_float, c_void_p, c_void_p, c_void_p, c_void_p, c_size_t, c_void_p]),
     "nb_kl_vp_jsd_combine": (c_int, [c_int64, c_int, c_void_p, c_void_p, c_int64, c_void_p, c_void_p, c_void_p,
                                      c_void_p, c_void_p]),
+    "nb_kl_gram": (c_int, [c_void_p, c_int64, c_int64, c_void_p, c_void_p, c_void_p]),
+    "nb_kl_project": (c_int, [c_void_p, c_int64, c_int64, c_void_p, c_int64, c_void_p, c_void_p, c_void_p]),
     "nb_kl_backward": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_float, c_float,
                                c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_int, c_void_p,
                                c_size_t, c_void_p]),

@@ -114,6 +114,7 @@ struct GemmProb {
   int k_dyn, K;            // k_dyn: K = round_up(n_valid, 128) (else K)
   int out_row0;            // output-map row of tile row 0
   int accumulate;          // 1: out += acc (TMA reduce-add), 0: out = acc (TMA store)
+  int out_bf16;            // 1: out is bf16 (32 x 32 boxes, 64-byte swizzle), stored rounded to nearest even
 };
 
 struct GemmArgs {

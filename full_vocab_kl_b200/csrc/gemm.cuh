@@ -155,6 +155,8 @@ __device__ __forceinline__ void gemm_mma(const GemmArgs& p, int nv, const SweepS
 // Each epilogue warp owns 32 output rows x 128 columns of the pair tile; it moves them in
 // 32 x 32 fp32 chunks: TMEM -> registers -> its staging buffer (128-byte swizzle: 16-byte
 // piece c of row r sits at piece c ^ (r & 7)) -> one TMA store (or TMA add) per chunk.
+// A bf16 output is rounded to nearest even and staged as 64-byte rows (64-byte swizzle:
+// piece c of row r at c ^ ((r >> 1) & 3)).
 __device__ __forceinline__ void gemm_epilogue(const GemmMaps& maps, const GemmArgs& p, int nv, const SweepSmem& s,
                                               uint32_t tmem_base, const WaitCtl& w) {
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
@@ -164,6 +166,7 @@ __device__ __forceinline__ void gemm_epilogue(const GemmMaps& maps, const GemmAr
   const uint32_t lane_addr = uint32_t(qq * 32) << 16;
   uint8_t* stage = s.out + (warp - kEpiWarp0) * kStageOutBytes;
   uint8_t* stage_row = stage + lane * 128;
+  uint8_t* stage_row16 = stage + lane * 64;
   bool staged = false;
   int acc = 0;
   uint32_t acc_phase = 0;
@@ -191,10 +194,23 @@ __device__ __forceinline__ void gemm_epilogue(const GemmMaps& maps, const GemmAr
       if (c0 >= q.N || row0 >= ti.M) continue;
       if (staged && lane == 0) bulk_wait_read();
       __syncwarp();
+      if (q.out_bf16) {
+        uint32_t packed[16];
 #pragma unroll
-      for (int c = 0; c < 8; ++c)
-        *reinterpret_cast<float4*>(stage_row + ((c ^ (lane & 7)) * 16)) =
-            make_float4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
+        for (int j = 0; j < 16; ++j) {
+          __nv_bfloat162 h2 = __floats2bfloat162_rn(v[2 * j], v[2 * j + 1]);
+          packed[j] = *reinterpret_cast<uint32_t*>(&h2);
+        }
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+          *reinterpret_cast<uint4*>(stage_row16 + ((c ^ ((lane >> 1) & 3)) * 16)) =
+              make_uint4(packed[4 * c], packed[4 * c + 1], packed[4 * c + 2], packed[4 * c + 3]);
+      } else {
+#pragma unroll
+        for (int c = 0; c < 8; ++c)
+          *reinterpret_cast<float4*>(stage_row + ((c ^ (lane & 7)) * 16)) =
+              make_float4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
+      }
       fence_async_smem();
       __syncwarp();
       if (lane == 0) {

@@ -850,6 +850,82 @@ nb_status nb_kl_forward_noalloc(const nb_kl_shape* shape, const void* h_s, const
                        n_valid, ws, size_t(NB_KL_NOALLOC_SCRATCH_BYTES), stream);
 }
 
+nb_status nb_kl_gram(const void* X, int64_t rows, int64_t d, float* G, void* workspace, void* stream) {
+  g_launches = 0;
+  if (!X || !G || !workspace) return NB_ERR_INVALID_ARG;
+  if (rows < 1 || d < 8 || d % 8 || rows > (int64_t(1) << 30) || d > 65536) return NB_ERR_INVALID_ARG;
+  if (!aligned16(X) || !aligned16(G) || !aligned16(workspace)) return NB_ERR_INVALID_ARG;
+  DevInfo dev;
+  nb_status s = device_info(dev);
+  if (s != NB_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  Ctrl* ctrl = static_cast<Ctrl*>(workspace);
+  if (cudaMemsetAsync(ctrl, 0, kCtrlBytes, st) != cudaSuccess) return NB_ERR_CUDA;
+  GemmMaps gm;
+  std::memset(&gm, 0, sizeof(gm));
+  // A = X^T (M = d contiguous) and B = X as K x N: both MN-major views of X's rows
+  bool ok = make_map(&gm.a[0], X, uint64_t(d), uint64_t(rows), uint64_t(d) * 2, 64, 64);
+  ok &= make_map(&gm.b[0], X, uint64_t(d), uint64_t(rows), uint64_t(d) * 2, 64, 64);
+  ok &= make_out_map(&gm.out[0], G, uint64_t(d), uint64_t(d));
+  if (!ok) return NB_ERR_CUDA;
+  GemmArgs g;
+  std::memset(&g, 0, sizeof(g));
+  g.nprob = 1;
+  g.n_valid = &ctrl->n_valid;
+  g.status = &ctrl->status;
+  g.wait_limit_ns = kWaitLimitNs;
+  GemmProb& q = g.prob[0];
+  q.a_mn = 1;
+  q.b_mn = 1;
+  q.M = int(d);
+  q.N = int(d);
+  q.K = int(rows);
+  const int tiles = int((d + kPairM - 1) / kPairM * ((d + kBlockN - 1) / kBlockN));
+  next_cat(NB_KL_KERNEL_GEMM_BWD);
+  launch(gemm_kernel, dim3(pair_grid(dev, tiles)), dim3(kThreads), size_t(kSmemBytes), st, gm, g);
+  return check_launch();
+}
+
+nb_status nb_kl_project(const void* X, int64_t rows, int64_t d, const void* B, int64_t k, void* Y, void* workspace,
+                        void* stream) {
+  g_launches = 0;
+  if (!X || !B || !Y || !workspace) return NB_ERR_INVALID_ARG;
+  if (rows < 1 || d < 8 || k < 8 || d % 8 || k % 8) return NB_ERR_INVALID_ARG;
+  if (rows > (int64_t(1) << 30) || d > 65536 || k > 65536) return NB_ERR_INVALID_ARG;
+  if (!aligned16(X) || !aligned16(B) || !aligned16(Y) || !aligned16(workspace)) return NB_ERR_INVALID_ARG;
+  DevInfo dev;
+  nb_status s = device_info(dev);
+  if (s != NB_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  Ctrl* ctrl = static_cast<Ctrl*>(workspace);
+  if (cudaMemsetAsync(ctrl, 0, kCtrlBytes, st) != cudaSuccess) return NB_ERR_CUDA;
+  GemmMaps gm;
+  std::memset(&gm, 0, sizeof(gm));
+  // A = X (K-major rows), B = the basis [d][k] as K x N (MN-major), out = Y [rows][k] bf16
+  bool ok = make_map(&gm.a[0], X, uint64_t(d), uint64_t(rows), uint64_t(d) * 2, kBlockK, kBlockM);
+  ok &= make_map(&gm.b[0], B, uint64_t(k), uint64_t(d), uint64_t(k) * 2, 64, 64);
+  ok &= make_map(&gm.out[0], Y, uint64_t(k), uint64_t(rows), uint64_t(k) * 2, 32, 32, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
+                 CU_TENSOR_MAP_SWIZZLE_64B);
+  if (!ok) return NB_ERR_CUDA;
+  GemmArgs g;
+  std::memset(&g, 0, sizeof(g));
+  g.nprob = 1;
+  g.n_valid = &ctrl->n_valid;
+  g.status = &ctrl->status;
+  g.wait_limit_ns = kWaitLimitNs;
+  GemmProb& q = g.prob[0];
+  q.a_mn = 0;
+  q.b_mn = 1;
+  q.M = int(rows);
+  q.N = int(k);
+  q.K = int(d);
+  q.out_bf16 = 1;
+  const int tiles = int((rows + kPairM - 1) / kPairM * ((k + kBlockN - 1) / kBlockN));
+  next_cat(NB_KL_KERNEL_GEMM_BWD);
+  launch(gemm_kernel, dim3(pair_grid(dev, tiles)), dim3(kThreads), size_t(kSmemBytes), st, gm, g);
+  return check_launch();
+}
+
 nb_status nb_kl_debug_gemm(const void* A, int a_mn_major, const void* B, int b_mn_major, int64_t M, int64_t N,
                            int64_t K, float* C, void* workspace, void* stream) {
   g_launches = 0;

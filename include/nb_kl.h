@@ -158,6 +158,30 @@ NB_KL_API nb_status nb_kl_vp_jsd_combine(int64_t n_tokens, int n_parts, const fl
                                const int64_t* labels, int64_t ignore_index, float* loss_tok, float* aux,
                                float* loss_mean, int64_t* n_valid, void* stream);
 
+/* ---- Spectral-compression front end ----------------------------------------------------
+ * "Nitrobrew tweet analysis": thread item 6/8 (spectral compression shrinks the hidden state
+ * below d_model, no longer exactly) and the evaluation table's "SVD-Nitrobrew" row (k floats
+ * per token). With the thin SVD W_t = U S V^T and V_k the right singular vectors of the k
+ * largest singular values, the teacher sends h_t' = V_k^T h_t and the loss uses
+ * W_t' = W_t V_k = U_k S_k with d_t = k: its teacher logits are those of the best rank-k
+ * approximation of W_t. Both products are nb_kl_project; V_k comes from the eigenvectors of
+ * the Gram matrix nb_kl_gram(W_t) (the small d_t x d_t eigendecomposition is the caller's,
+ * once per teacher checkpoint). Both run on the same tcgen05 GEMM as the backward.
+ *
+ * Workspace of both calls: NB_KL_SMALL_WORKSPACE_BYTES of device memory (status word), 16-byte
+ * aligned; nb_kl_device_status reads it. Pointers are device pointers, 16-byte aligned. */
+#define NB_KL_SMALL_WORKSPACE_BYTES 256
+
+/* G = X^T X: X [rows, d] bf16 row-major, G [d, d] fp32 (overwritten; fp32 accumulation).
+ * d a multiple of 8, 8 <= d <= 65536, 1 <= rows <= 2^30. */
+NB_KL_API nb_status nb_kl_gram(const void* X, int64_t rows, int64_t d, float* G, void* workspace, void* stream);
+
+/* Y = X B: X [rows, d] bf16, B [d, k] bf16 (row-major: k contiguous), Y [rows, k] bf16, the
+ * fp32 sum rounded to nearest even. d and k multiples of 8 (>= 8, <= 65536). Teacher codes
+ * (X = h_t, B = V_k) and the compressed unembedding (X = W_t, B = V_k). */
+NB_KL_API nb_status nb_kl_project(const void* X, int64_t rows, int64_t d, const void* B, int64_t k, void* Y,
+                        void* workspace, void* stream);
+
 /* Backward ("仓库实现": recompute the logit blocks; gradients reach h_s and W_s only).
  * Inputs lse_s, lse_t, aux are the forward's outputs for the same arguments; grad_out is
  * one fp32 on the device (dOut/dloss_mean). Writes dh_s [n_tokens, d_s] (masked rows 0)

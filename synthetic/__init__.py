@@ -13,6 +13,8 @@ from .workloads import (  # noqa: F401
     Workload,
     bf16_bits_to_f32,
     f32_to_bf16_bits,
+    gaussian_bf16,
+    matrix_with_spectrum,
     make_inputs,
     make_custom,
 )

@@ -41,7 +41,7 @@ import numpy as np
 IGNORE_INDEX = -100
 
 # tensor ids of the per-tensor random streams
-_ID_HS, _ID_HT, _ID_WS, _ID_WT, _ID_EPS, _ID_Q, _ID_MASK, _ID_LABEL, _ID_BOOST, _ID_DW = range(10)
+_ID_HS, _ID_HT, _ID_WS, _ID_WT, _ID_EPS, _ID_Q, _ID_MASK, _ID_LABEL, _ID_BOOST, _ID_DW, _ID_SPEC = range(11)
 _BLOCK_ROWS = 8192
 
 
@@ -324,3 +324,20 @@ def make_custom(N: int, d_s: int, d_t: int, V: int, beta: float, tau: float, *, 
                  h_dtype=h_dtype, teacher=teacher, mask=mask, masked_per_seq=n_masked,
                  boost_frac=boost_frac, boost=boost, accumulate_dW=accumulate_dW)
     return make_inputs(w, seed)
+
+
+def matrix_with_spectrum(rows: int, cols: int, sigma, seed: int = 0) -> np.ndarray:
+    """bf16 bits of U diag(sigma) Q^T with random orthonormal U [rows, cols] and Q [cols, cols]
+    (QR of seeded Gaussians), for tests of a rank-k teacher basis. sigma has `cols` entries."""
+    sigma = np.asarray(sigma, dtype=np.float64)
+    if sigma.shape != (cols,):
+        raise ValueError("sigma needs one value per column")
+    g = _rng(seed, _ID_SPEC)
+    U, _ = np.linalg.qr(g.standard_normal((rows, cols)))
+    Q, _ = np.linalg.qr(g.standard_normal((cols, cols)))
+    return f32_to_bf16_bits(((U * sigma) @ Q.T).astype(np.float32))
+
+
+def gaussian_bf16(rows: int, cols: int, std: float, seed: int = 0, stream: int = _ID_SPEC) -> np.ndarray:
+    """bf16 bits of a seeded N(0, std^2) matrix (row blocks drawn in parallel)."""
+    return _normal_rows_bf16(seed, stream, rows, cols, std)

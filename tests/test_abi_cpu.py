@@ -153,3 +153,15 @@ def test_vocab_parallel_argument_errors(L):
                                     p[8], wsb, None) == L.NB_ERR_INVALID_ARG
     assert lib.nb_kl_vp_jsd_combine(256, 2, None, p[1], -100, p[2], p[3], p[4], p[5],
                                     None) == L.NB_ERR_INVALID_ARG
+
+
+def test_spectral_argument_errors(L):
+    lib = L.lib()
+    p = [ctypes.c_void_p(v) for v in FAKE]
+    # d not a multiple of 8, rows < 1, misaligned output, k < 8
+    assert lib.nb_kl_gram(p[0], 100, 12, p[1], p[2], None) == L.NB_ERR_INVALID_ARG
+    assert lib.nb_kl_gram(p[0], 0, 64, p[1], p[2], None) == L.NB_ERR_INVALID_ARG
+    assert lib.nb_kl_gram(p[0], 100, 64, ctypes.c_void_p(FAKE[1] + 4), p[2], None) == L.NB_ERR_INVALID_ARG
+    assert lib.nb_kl_project(p[0], 100, 64, p[1], 4, p[2], p[3], None) == L.NB_ERR_INVALID_ARG
+    assert lib.nb_kl_project(p[0], 100, 64, None, 64, p[2], p[3], None) == L.NB_ERR_INVALID_ARG
+    assert lib.nb_kl_project(p[0], 100, 60, p[1], 64, p[2], p[3], None) == L.NB_ERR_INVALID_ARG
