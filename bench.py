@@ -59,16 +59,19 @@ def measured_peaks():
     return dict(FALLBACK), "fallback"
 
 
-def algorithmic_flops(w, n_valid):
+def algorithmic_flops(w, n_valid, V=None, proj=0.0):
     """FLOPs of the method on valid rows: forward sweep, [JSD second sweep], recompute sweep,
-    dh_s and dW_s products."""
-    sweep = 2.0 * n_valid * w.V * (w.d_s + w.d_t)
+    dh_s and dW_s products (V: the vocabulary rows this rank holds), and the teacher-code
+    projection of the spectral front end (`proj`, all positions)."""
+    V = w.V if V is None else V
+    sweep = 2.0 * n_valid * V * (w.d_s + w.d_t)
     jsd = 0.0 < w.beta < 1.0
     return {
         "sweep_fwd": sweep,
         "sweep_jsd": sweep if jsd else 0.0,
         "sweep_grad": sweep,
-        "gemm_bwd": 4.0 * n_valid * w.V * w.d_s,
+        "gemm_bwd": 4.0 * n_valid * V * w.d_s,
+        "gemm_proj": proj,
     }
 
 
@@ -86,16 +89,20 @@ def kernel_source_sha():
     return h.hexdigest()[:16]
 
 
-def profiled_traffic(kernel: str, workload: str):
+def profiled_traffic(kernel: str, workload: str, chunk_v: int):
     """Per-launch DRAM bytes (read + write) of `kernel` from the committed full-size ncu summary
-    of the workload, if that summary was taken from the current device code."""
+    of the workload, if that summary was taken from the current device code with the same
+    backward chunk (the per-launch traffic of the backward kernels scales with it)."""
     p = os.path.join(ROOT, "profiles", f"fullsize_{workload}.md")
     if not os.path.exists(p):
         return None
     txt = open(p).read()
     m_sha = re.search(r"kernel_source_sha:\s*([0-9a-f]+)", txt)
     m_tr = re.search(re.escape(kernel) + r"\.dram_bytes_per_launch:\s*([0-9.eE+]+)", txt)
+    m_ch = re.search(r"chunk_columns:\s*([0-9]+)", txt)
     if not m_sha or not m_tr or m_sha.group(1) != kernel_source_sha():
+        return None
+    if not m_ch or int(m_ch.group(1)) != chunk_v:
         return None
     return float(m_tr.group(1))
 
@@ -286,25 +293,109 @@ def run_library(args):
 
     h_s, h_t, W_s, W_t = (to_dev(getattr(x, k)) for k in ("h_s", "h_t", "W_s", "W_t"))
     labels = torch.from_numpy(x.labels).to(dev)
-    shape = nb.make_shape(h_s, W_s, h_t, W_t, labels, chunk_v=args.chunk_v)
-    ws_bytes = nb.workspace_bytes(shape, w.beta)
-    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
     N = labels.shape[0]
     f32 = dict(dtype=torch.float32, device=dev)
+    lib = _abi.lib()
+    grad_out = torch.ones((), **f32)
+    V_rank, proj_flops, mode_cfg = w.V, 0.0, {}
+
+    if args.front_end:
+        # spectral front end: a full-width teacher (Gaussian unembedding, RMS-normalised hidden
+        # states, drawn on the device from a seeded generator) compressed to the workload's rank
+        from full_vocab_kl_b200 import spectral
+        gen = torch.Generator(device=dev)
+        gen.manual_seed(1000 + rank)
+        d_full = args.teacher_width
+        W_full = (torch.randn((w.V, d_full), generator=gen, device=dev) * (w.w_std / d_full ** 0.5)).to(
+            torch.bfloat16)
+        h_full = torch.randn((N, d_full), generator=gen, device=dev)
+        h_full = (h_full / (h_full.pow(2).mean(1, keepdim=True) + 1e-6).sqrt()).to(torch.bfloat16)
+        basis = spectral.spectral_factor(W_full, w.d_t)
+        W_t = basis.W_code
+        code = torch.empty((N, w.d_t), dtype=torch.bfloat16, device=dev)
+        h_t = h_full
+        del W_full
+        proj_flops = 2.0 * N * d_full * w.d_t
+        mode_cfg = {"front_end": "spectral", "teacher_width": d_full, "rank": w.d_t}
+
+    if args.vocab_parallel:
+        from full_vocab_kl_b200.vocab_parallel import LibraryKernels, shard_range, vp_backward, vp_forward
+        v0, v1 = shard_range(w.V, rank, world)
+        W_s, W_t = W_s[v0:v1].contiguous(), W_t[v0:v1].contiguous()
+        V_rank = v1 - v0
+        mode_cfg.update({"vocab_shard_rows": V_rank})
+
+        class CountingKernels(LibraryKernels):
+            launches = 0
+
+            def _count(self, r):
+                CountingKernels.launches += lib.nb_kl_last_launch_count()
+                return r
+
+            def state(self, *a, **k):
+                return self._count(super().state(*a, **k))
+
+            def combine(self, *a, **k):
+                return self._count(super().combine(*a, **k))
+
+            def jsd_partial(self, *a, **k):
+                return self._count(super().jsd_partial(*a, **k))
+
+            def jsd_combine(self, *a, **k):
+                return self._count(super().jsd_combine(*a, **k))
+
+            def backward(self, *a, **k):
+                return self._count(super().backward(*a, **k))
+
+        kern = CountingKernels()
+        gather = (lambda t: t[None].contiguous()) if world == 1 else None
+        reduce = (lambda t: t) if world == 1 else None
+        vp_ws = {}
+
+    if args.handoff:
+        # the teacher's hidden rows arrive through the hand-off copy (valid rows only) into a
+        # local buffer that the loss then reads; the buffer passed to `step` stands for the
+        # teacher's memory (another GPU's, or an IPC mapping, in a two-GPU deployment)
+        from full_vocab_kl_b200 import handoff
+        ht_local = torch.zeros_like(h_t)
+        handoff_bytes = n_valid * h_t.shape[1] * h_t.element_size()
+        mode_cfg["handoff_bytes_per_step"] = handoff_bytes
+
+    shape = nb.make_shape(h_s, W_s, code if args.front_end else h_t, W_t, labels, chunk_v=args.chunk_v)
+    ws_bytes = nb.workspace_bytes(shape, w.beta)
+    ws = None if args.vocab_parallel else torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
     out = {"loss_tok": torch.empty(N, **f32), "lse_s": torch.empty(N, **f32), "lse_t": torch.empty(N, **f32),
            "aux": torch.empty(N, **f32), "loss_mean": torch.empty((), **f32),
            "n_valid": torch.empty((), dtype=torch.int64, device=dev)}
+    if args.side:
+        out["entropy_s"] = torch.empty(N, **f32)
+        out["logp_label"] = torch.empty(N, **f32)
     dh = torch.empty((N, w.d_s), **f32)
-    dW = torch.zeros((w.V, w.d_s), **f32) if w.accumulate_dW else torch.empty((w.V, w.d_s), **f32)
-    grad_out = torch.ones((), **f32)
-    lib = _abi.lib()
+    dW = torch.zeros((V_rank, w.d_s), **f32) if w.accumulate_dW else torch.empty((V_rank, w.d_s), **f32)
 
     def step(hs, ht, lab):
-        nb.kl_forward(hs, W_s, ht, W_t, lab, w.beta, w.tau, workspace=ws, out=out, chunk_v=args.chunk_v)
+        if args.vocab_parallel:
+            CountingKernels.launches = 0
+            f = vp_forward(hs, W_s, ht, W_t, lab, w.beta, w.tau, vocab_offset=v0, side=args.side, kernels=kern,
+                           all_gather=gather)
+            vp_backward(hs, W_s, ht, W_t, lab, w.beta, w.tau, f["lse_s"], f["lse_t"], f["aux"], grad_out,
+                        kernels=kern, workspace=f["workspace"], all_reduce=reduce)
+            out["loss_mean"], out["n_valid"] = f["loss_mean"], f["n_valid"]
+            return CountingKernels.launches
+        n0 = 0
+        if args.handoff:
+            ht = handoff.receive_rows(ht, lab, out=ht_local)
+            n0 += lib.nb_kl_last_launch_count()
+        if args.front_end:
+            spectral.project(ht, basis.V_k, out=code)
+            n0 += lib.nb_kl_last_launch_count()
+            ht = code
+        nb.kl_forward(hs, W_s, ht, W_t, lab, w.beta, w.tau, workspace=ws, out=out, chunk_v=args.chunk_v,
+                      side=args.side)
         n1 = lib.nb_kl_last_launch_count()
         nb.kl_backward(hs, W_s, ht, W_t, lab, w.beta, w.tau, out["lse_s"], out["lse_t"], out["aux"], grad_out,
                        dh_s=dh, dW_s=dW, accumulate_dW=w.accumulate_dW, workspace=ws, chunk_v=args.chunk_v)
-        return n1 + lib.nb_kl_last_launch_count()
+        return n0 + n1 + lib.nb_kl_last_launch_count()
 
     stream = torch.cuda.current_stream(dev)
     for _ in range(args.warmup):
@@ -326,9 +417,10 @@ def run_library(args):
     e1.record(stream)
     barrier()
     lib.nb_kl_timing_enable(0)
-    ms_arr = (ctypes.c_double * 5)()
-    cnt_arr = (ctypes.c_int * 5)()
-    lib.nb_kl_timing_read(ctypes.cast(ms_arr, ctypes.c_void_p), ctypes.cast(cnt_arr, ctypes.c_void_p), 5)
+    ncat = len(_abi.KERNEL_CATEGORIES)
+    ms_arr = (ctypes.c_double * ncat)()
+    cnt_arr = (ctypes.c_int * ncat)()
+    lib.nb_kl_timing_read(ctypes.cast(ms_arr, ctypes.c_void_p), ctypes.cast(cnt_arr, ctypes.c_void_p), ncat)
     clk = clocks.stop() if rank == 0 else None
     ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
     peak_extra = torch.cuda.max_memory_allocated(dev) - mem0
@@ -368,25 +460,36 @@ def run_library(args):
     if rank == 0:
         ms_step = ms / args.steps
         tokens = N * world
-        value = whole_job_rate(N, world, ms_step)
-        flops = algorithmic_flops(w, n_valid)
-        step_flops = sum(flops.values())
+        # vocabulary-parallel ranks share one batch (strong scaling); otherwise each rank runs its own
+        units = N if args.vocab_parallel else N * world
+        value = units / (ms_step * 1e-3)
+        flops = algorithmic_flops(w, n_valid, V=V_rank, proj=proj_flops)
+        step_flops = sum(flops.values()) * world
         tflops = step_flops / (ms_step * 1e-3) / 1e12
         peaks, peak_src = measured_peaks()
         cats = _abi.KERNEL_CATEGORIES
         kms = {c: ms_arr[i] / args.steps for i, c in enumerate(cats)}
         kcount = {c: cnt_arr[i] / args.steps for i, c in enumerate(cats)}
-        dom = max(("sweep_fwd", "sweep_jsd", "sweep_grad", "gemm_bwd"), key=lambda c: kms[c])
+        dom = max(("sweep_fwd", "sweep_jsd", "sweep_grad", "gemm_bwd", "gemm_proj"), key=lambda c: kms[c])
         per_launch_ms = kms[dom] / max(kcount[dom], 1)
         per_launch_flops = flops[dom] / max(kcount[dom], 1)
         achieved = per_launch_flops / (per_launch_ms * 1e-3) / 1e12
         peak = peaks.get("bf16_tflops_sustained", FALLBACK["bf16_tflops_sustained"])
-        traffic = profiled_traffic(dom, w.name)
+        chunk_cols = lib.nb_kl_chunk_columns(_abi.shape_ptr(shape))
+        traffic = (profiled_traffic(dom, w.name, chunk_cols)
+                   if not (args.vocab_parallel or args.front_end) else None)
+        config = workload_config(w, n_valid, world)
+        if args.vocab_parallel:
+            config["parallelism"] = f"vocab{world}"
+        if args.side:
+            config["side_outputs"] = True
+        config.update(mode_cfg)
         result = {
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+            "scaling": "strong" if args.vocab_parallel else "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded; shapes of the workload)",
-            "config": workload_config(w, n_valid, world),
+            "config": config,
             "tflops": tflops, "pct_bf16_peak_datasheet": 100.0 * tflops / DATASHEET_BF16_TFLOPS,
             "pct_bf16_peak_measured": 100.0 * tflops / peaks.get("bf16_tflops", FALLBACK["bf16_tflops"]),
             "roofline": {"bound": "tensor", "kernel": dom, "achieved": achieved, "peak": peak,
@@ -395,17 +498,21 @@ def run_library(args):
                          "algorithmic_flops_per_launch": per_launch_flops, "launch_ms": per_launch_ms},
             "kernel_ms_per_step": kms, "kernel_launches_per_step": kcount,
             "kernel_tflops": {c: (flops[c] / (kms[c] * 1e-3) / 1e12 if kms[c] > 0 else None)
-                              for c in ("sweep_fwd", "sweep_jsd", "sweep_grad", "gemm_bwd")},
-            "e2e": {"value": whole_job_rate(N, world, ms_e2e / e2e_steps), "unit": "tokens/s",
+                              for c in ("sweep_fwd", "sweep_jsd", "sweep_grad", "gemm_bwd", "gemm_proj")},
+            "e2e": {"value": units / (ms_e2e / e2e_steps * 1e-3), "unit": "tokens/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps},
             "gpu_launches": launches,
+            **({"handoff": {"bytes_per_step": handoff_bytes, "ms_per_step": kms["handoff"],
+                            "gbs": (2.0 * handoff_bytes / (kms["handoff"] * 1e-3) / 1e9) if kms["handoff"] else None,
+                            "note": "read + write bytes over the copy's device time; one GPU: HBM to HBM"}}
+               if args.handoff else {}),
             "clocks": clk,
-            "scratch_bytes": ws_bytes, "peak_extra_alloc_bytes": int(peak_extra), "chunk_v": args.chunk_v,
+            "scratch_bytes": ws_bytes, "peak_extra_alloc_bytes": int(peak_extra), "chunk_v": chunk_cols,
         }
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
-    if rank == 0 and not args.no_cpu_baseline:
+    if rank == 0 and not args.no_cpu_baseline and not args.front_end:
         result["cpu_baseline"] = cpu_baseline(x)
     if rank == 0:
         print(json.dumps(result), flush=True)
@@ -422,7 +529,19 @@ def main():
     ap.add_argument("--impl", default="library", choices=["library", "reference"])
     ap.add_argument("--chunk-v", type=int, default=0, help="backward vocabulary chunk (0: library default)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--side", action="store_true",
+                    help="forward with the student entropy / sampled-token log-prob side outputs")
+    ap.add_argument("--vocab-parallel", action="store_true",
+                    help="shard the unembeddings by rows over the ranks (one batch, strong scaling)")
+    ap.add_argument("--front-end", choices=["spectral"], default=None,
+                    help="time the teacher-code projection of a full-width teacher with the loss")
+    ap.add_argument("--handoff", action="store_true",
+                    help="the teacher's hidden rows reach the loss through the hand-off copy")
+    ap.add_argument("--teacher-width", type=int, default=4096,
+                    help="hidden width of the full teacher for --front-end spectral")
     args = ap.parse_args()
+    if sum(map(bool, (args.front_end, args.vocab_parallel, args.handoff))) > 1:
+        ap.error("--front-end, --vocab-parallel and --handoff are separate measurements")
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     if args.impl == "reference":

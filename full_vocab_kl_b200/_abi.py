@@ -28,6 +28,7 @@ SMALL_WORKSPACE_BYTES = 256   # NB_KL_SMALL_WORKSPACE_BYTES
 # every function the header declares, with (restype, argtypes)
 SIGNATURES = {
     "nb_kl_workspace_size": (c_size_t, [c_void_p, c_float]),
+    "nb_kl_chunk_columns": (c_int64, [c_void_p]),
     "nb_kl_forward": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_float, c_float,
                               c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_size_t,
                               c_void_p]),
@@ -44,6 +45,8 @@ SIGNATURES = {
                                      c_void_p, c_void_p]),
     "nb_kl_gram": (c_int, [c_void_p, c_int64, c_int64, c_void_p, c_void_p, c_void_p]),
     "nb_kl_project": (c_int, [c_void_p, c_int64, c_int64, c_void_p, c_int64, c_void_p, c_void_p, c_void_p]),
+    "nb_kl_handoff_rows": (c_int, [c_void_p, c_void_p, c_int64, c_int64, c_void_p, c_int64, c_void_p]),
+    "nb_kl_enable_peer_access": (c_int, [c_int]),
     "nb_kl_backward": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_float, c_float,
                                c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_int, c_void_p,
                                c_size_t, c_void_p]),
@@ -60,7 +63,7 @@ SIGNATURES = {
     "nb_kl_timing_read": (c_int, [c_void_p, c_void_p, c_int]),
 }
 
-KERNEL_CATEGORIES = ("sweep_fwd", "sweep_jsd", "sweep_grad", "gemm_bwd", "rowops")
+KERNEL_CATEGORIES = ("sweep_fwd", "sweep_jsd", "sweep_grad", "gemm_bwd", "rowops", "gemm_proj", "handoff")
 
 
 class Shape(ctypes.Structure):

@@ -92,10 +92,11 @@ bool make_layout(const nb_kl_shape* sh, float beta, Layout& L) {
   L.lda_t = int64_t(L.kb_t) * kBlockK * (L.split ? 2 : 1);
   L.n_vt = int((L.V + kBlockN - 1) / kBlockN);
   L.n_split = 2 * ((L.n_vt + kTilesPerUnitFwd - 1) / kTilesPerUnitFwd);  // two column halves per unit
-  // default chunk: about 4096 gradient tiles per sweep launch (the two gradient buffers then
-  // take ~0.5 GB whatever the token count), but at least 4 d_s columns so that the compacted
-  // dh accumulator is not re-added too often; between 2048 and 32768 columns
-  const int64_t by_tiles = (int64_t(1) << 20) / (L.N_pad / kBlockM);
+  // default chunk: about 8192 gradient tiles of 128 x 256 per sweep launch (the two gradient
+  // buffers then take ~1 GB whatever the token count; longer chunks mean fewer launches and
+  // fewer re-adds of the compacted dh accumulator), but at least 4 d_s columns; between 2048
+  // and 32768 columns
+  const int64_t by_tiles = (int64_t(1) << 21) / (L.N_pad / kBlockM);
   const int64_t auto_chunk =
       round_up(std::max<int64_t>(2048, std::min<int64_t>(32768, std::max<int64_t>(by_tiles, 4 * L.d_s))), kBlockN);
   L.chunk_v = sh->chunk_v ? sh->chunk_v : std::min<int64_t>(auto_chunk, round_up(L.V, kBlockN));
@@ -596,6 +597,12 @@ size_t nb_kl_workspace_size(const nb_kl_shape* shape, float beta) {
   return L.total;
 }
 
+int64_t nb_kl_chunk_columns(const nb_kl_shape* shape) {
+  Layout L;
+  if (!make_layout(shape, 1.0f, L)) return 0;
+  return L.chunk_v;
+}
+
 const char* nb_kl_status_string(nb_status s) {
   switch (s) {
     case NB_OK: return "ok";
@@ -881,7 +888,7 @@ nb_status nb_kl_gram(const void* X, int64_t rows, int64_t d, float* G, void* wor
   q.N = int(d);
   q.K = int(rows);
   const int tiles = int((d + kPairM - 1) / kPairM * ((d + kBlockN - 1) / kBlockN));
-  next_cat(NB_KL_KERNEL_GEMM_BWD);
+  next_cat(NB_KL_KERNEL_GEMM_PROJ);
   launch(gemm_kernel, dim3(pair_grid(dev, tiles)), dim3(kThreads), size_t(kSmemBytes), st, gm, g);
   return check_launch();
 }
@@ -921,9 +928,42 @@ nb_status nb_kl_project(const void* X, int64_t rows, int64_t d, const void* B, i
   q.K = int(d);
   q.out_bf16 = 1;
   const int tiles = int((rows + kPairM - 1) / kPairM * ((k + kBlockN - 1) / kBlockN));
-  next_cat(NB_KL_KERNEL_GEMM_BWD);
+  next_cat(NB_KL_KERNEL_GEMM_PROJ);
   launch(gemm_kernel, dim3(pair_grid(dev, tiles)), dim3(kThreads), size_t(kSmemBytes), st, gm, g);
   return check_launch();
+}
+
+nb_status nb_kl_handoff_rows(const void* src, void* dst, int64_t n_rows, int64_t row_bytes, const int64_t* labels,
+                             int64_t ignore_index, void* stream) {
+  g_launches = 0;
+  if (n_rows < 0 || row_bytes < 16 || row_bytes % 16 || row_bytes > (int64_t(1) << 24)) return NB_ERR_INVALID_ARG;
+  if (n_rows == 0) return NB_OK;
+  if (!src || !dst || !aligned16(src) || !aligned16(dst)) return NB_ERR_INVALID_ARG;
+  DevInfo dev;
+  nb_status s = device_info(dev);
+  if (s != NB_OK) return s;
+  // two resident 256-thread blocks per SM; fewer when there are fewer rows than warps
+  const long long warps = std::min<long long>(n_rows, 16ll * dev.sms);
+  const unsigned blocks = unsigned((warps + 7) / 8);
+  next_cat(NB_KL_KERNEL_HANDOFF);
+  launch(handoff_rows_kernel, dim3(blocks), dim3(256), 0, static_cast<cudaStream_t>(stream),
+         static_cast<const uint4*>(src), static_cast<uint4*>(dst), (long long)n_rows, (long long)(row_bytes / 16),
+         labels, (long long)ignore_index);
+  return check_launch();
+}
+
+nb_status nb_kl_enable_peer_access(int peer_device) {
+  int dev = 0, can = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return NB_ERR_CUDA;
+  if (peer_device == dev) return NB_OK;
+  if (cudaDeviceCanAccessPeer(&can, dev, peer_device) != cudaSuccess) return NB_ERR_INVALID_ARG;
+  if (!can) return NB_ERR_UNSUPPORTED;
+  const cudaError_t e = cudaDeviceEnablePeerAccess(peer_device, 0);
+  if (e == cudaErrorPeerAccessAlreadyEnabled) {
+    cudaGetLastError();   // the call also recorded it as the last error: clear that
+    return NB_OK;
+  }
+  return e == cudaSuccess ? NB_OK : NB_ERR_CUDA;
 }
 
 nb_status nb_kl_debug_gemm(const void* A, int a_mn_major, const void* B, int b_mn_major, int64_t M, int64_t N,

@@ -343,6 +343,34 @@ __global__ void __launch_bounds__(1024)
   }
 }
 
+// ------------------------------------------------------------------ hand-off of hidden rows
+// dst row r = src row r for every row whose label is not ignore_index (all rows without
+// labels); rows are row_vecs 16-byte vectors. src may be another GPU's memory (a peer or
+// IPC mapping): each warp copies one row at a time with four independent 16-byte loads in
+// flight per lane, so that many requests cover the link latency; rows are strided over all
+// warps of the grid.
+__global__ void __launch_bounds__(256)
+    handoff_rows_kernel(const uint4* __restrict__ src, uint4* __restrict__ dst, long long n_rows,
+                        long long row_vecs, const int64_t* __restrict__ labels, long long ignore_index) {
+  const long long warp_id = (blockIdx.x * 256ll + threadIdx.x) >> 5;
+  const long long n_warps = (long long)gridDim.x * 8;
+  const int lane = threadIdx.x & 31;
+  for (long long r = warp_id; r < n_rows; r += n_warps) {
+    if (labels && labels[r] == ignore_index) continue;
+    const uint4* s = src + r * row_vecs;
+    uint4* d = dst + r * row_vecs;
+    long long c = lane;
+    for (; c + 96 < row_vecs; c += 128) {
+      const uint4 a = s[c], b = s[c + 32], e = s[c + 64], f = s[c + 96];
+      d[c] = a;
+      d[c + 32] = b;
+      d[c + 64] = e;
+      d[c + 96] = f;
+    }
+    for (; c < row_vecs; c += 32) d[c] = s[c];
+  }
+}
+
 // Deterministic masked mean: fixed-order fp64 sum of loss_tok (masked rows hold 0).
 __global__ void __launch_bounds__(1024) mean_kernel(const float* __restrict__ loss_tok, int N,
                                                     const Ctrl* __restrict__ ctrl, float* loss_mean) {

@@ -77,6 +77,11 @@ typedef struct nb_kl_shape {
  * Returns 0 for an invalid shape. */
 NB_KL_API size_t nb_kl_workspace_size(const nb_kl_shape* shape, float beta);
 
+/* Vocabulary columns per backward chunk for this shape: shape->chunk_v, or the library's
+ * default when it is 0 (about 8192 gradient tiles of 128 x 256 per launch, at least 4 d_s,
+ * between 2048 and 32768, at most the vocabulary rounded up to 256). 0 for an invalid shape. */
+NB_KL_API int64_t nb_kl_chunk_columns(const nb_kl_shape* shape);
+
 /* Forward ("Nitrobrew 的两个动作": block GEMMs + online log-sum-exp + KL numerator).
  * Outputs (device, caller-owned): loss_tok, lse_s, lse_t, aux [n_tokens] fp32 —
  * lse_* are natural-log LSEs of the tempered logits u = z / tau; aux is the per-token KL
@@ -182,6 +187,25 @@ NB_KL_API nb_status nb_kl_gram(const void* X, int64_t rows, int64_t d, float* G,
 NB_KL_API nb_status nb_kl_project(const void* X, int64_t rows, int64_t d, const void* B, int64_t k, void* Y,
                         void* workspace, void* stream);
 
+/* ---- Teacher -> student hand-off of hidden states -----------------------------------------
+ * "Nitrobrew tweet analysis", thread items 3/8 and 4/8 and section "OPD 为什么更痛": when teacher
+ * and student sit on different GPUs, what must cross to the loss is the teacher's final hidden
+ * state (d_t values per token, or the rank-k code) instead of V logits. src is the teacher's
+ * [n_rows, row_bytes] buffer as this process sees it: another GPU's memory reached through peer
+ * access (nb_kl_enable_peer_access) or a CUDA IPC mapping, or local memory. The kernel reads it
+ * with plain 16-byte loads (no TMA, no multicast) and writes dst (local, [n_rows, row_bytes]);
+ * with labels (device int64 [n_rows]) only rows whose label is not ignore_index cross the link
+ * and the other dst rows keep their contents. Both pointers 16-byte aligned, row_bytes a
+ * multiple of 16. The loss can also take src directly as h_t: its row gather then reads the
+ * valid rows over the link in each call (forward and backward), where one hand-off into local
+ * memory reads them once. */
+NB_KL_API nb_status nb_kl_handoff_rows(const void* src, void* dst, int64_t n_rows, int64_t row_bytes,
+                             const int64_t* labels, int64_t ignore_index, void* stream);
+
+/* Enable this device's access to peer_device's memory (cudaDeviceEnablePeerAccess; already
+ * enabled is not an error). NB_ERR_UNSUPPORTED when the devices cannot reach each other. */
+NB_KL_API nb_status nb_kl_enable_peer_access(int peer_device);
+
 /* Backward ("仓库实现": recompute the logit blocks; gradients reach h_s and W_s only).
  * Inputs lse_s, lse_t, aux are the forward's outputs for the same arguments; grad_out is
  * one fp32 on the device (dOut/dloss_mean). Writes dh_s [n_tokens, d_s] (masked rows 0)
@@ -246,7 +270,9 @@ enum {
   NB_KL_KERNEL_SWEEP_GRAD = 2,  /* backward recompute sweep writing the gradient chunk */
   NB_KL_KERNEL_GEMM_BWD = 3,    /* backward dh_s / dW_s GEMMs */
   NB_KL_KERNEL_ROWOPS = 4,      /* compaction, merges, mean */
-  NB_KL_KERNEL_CATEGORIES = 5
+  NB_KL_KERNEL_GEMM_PROJ = 5,   /* spectral front end: Gram and projection GEMMs */
+  NB_KL_KERNEL_HANDOFF = 6,     /* hand-off copy of hidden rows */
+  NB_KL_KERNEL_CATEGORIES = 7
 };
 
 /* Per calling thread: when on, every launch is bracketed by two CUDA events recorded on

@@ -108,6 +108,10 @@ PROFILE_WORKLOADS = {
         "opd_0p6b_4b_prof", 1, 640, 1024, 2560, 75776, 1.0, 1.0, 3.0,
         teacher="correlated", mask="prefix", masked_per_seq=128,
         description="profiling size of opd_0p6b_4b: 640 tokens (512 valid), V 75776"),
+    "spectral_prof": Workload(
+        "spectral_prof", 2, 4096, 4096, 512, 32768, 1.0, 1.0, 3.0,
+        teacher="spectral", mask="random", masked_per_seq=1434,
+        description="profiling size of spectral: 8192 tokens, V 32768, rank-512 teacher code"),
 }
 
 

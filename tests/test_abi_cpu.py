@@ -165,3 +165,15 @@ def test_spectral_argument_errors(L):
     assert lib.nb_kl_project(p[0], 100, 64, p[1], 4, p[2], p[3], None) == L.NB_ERR_INVALID_ARG
     assert lib.nb_kl_project(p[0], 100, 64, None, 64, p[2], p[3], None) == L.NB_ERR_INVALID_ARG
     assert lib.nb_kl_project(p[0], 100, 60, p[1], 64, p[2], p[3], None) == L.NB_ERR_INVALID_ARG
+
+
+def test_chunk_columns(L):
+    lib = L.lib()
+    # default: ~8192 gradient tiles of 128 x 256 per launch, at least 4 d_s, in [2048, 32768]
+    assert lib.nb_kl_chunk_columns(L.shape_ptr(shape(L))) == 32768
+    assert lib.nb_kl_chunk_columns(L.shape_ptr(shape(L, N=32768, ds=4096, dt=512))) == 16384
+    assert lib.nb_kl_chunk_columns(L.shape_ptr(shape(L, N=65536, ds=256, dt=256))) == 4096
+    assert lib.nb_kl_chunk_columns(L.shape_ptr(shape(L, N=256, V=1000, ds=256, dt=256))) == 1024
+    # an explicit chunk is kept; an invalid shape gives 0
+    assert lib.nb_kl_chunk_columns(L.shape_ptr(shape(L, chunk=4096))) == 4096
+    assert lib.nb_kl_chunk_columns(L.shape_ptr(shape(L, ds=100))) == 0

@@ -1,0 +1,122 @@
+"""Teacher -> student hand-off of hidden rows ("Nitrobrew tweet analysis", thread items 3/8 and
+4/8: the teacher's final hidden state crosses to the loss instead of V logits per token).
+
+A byte copy: results must be bit-exact. The two-process test shares the teacher's buffer
+through CUDA IPC (a CUDA tensor sent through a torch.multiprocessing queue); every gpurun call
+has one GPU, so both processes use it: the transfer is then an HBM copy, the code path (an IPC
+mapping read by plain loads) is the one a second GPU would use over NVLink. The processes do
+not wait on each other inside kernels: the hand-over is a host queue and a host event, both
+with timeouts.
+"""
+
+import subprocess
+
+import numpy as np
+import pytest
+
+import gpu_util as gu
+from synthetic import make_custom, make_inputs
+
+pytestmark = pytest.mark.gpu
+
+
+def _bits(t):
+    import torch
+    return t.view(torch.int16).cpu().numpy() if t.dtype == torch.bfloat16 else t.cpu().numpy()
+
+
+@pytest.mark.parametrize("N,d", [(1000, 2560), (1, 8), (37, 136), (4096, 520)])
+def test_all_rows_bit_exact(N, d):
+    import torch
+    from full_vocab_kl_b200 import handoff
+    g = torch.Generator(device="cuda")
+    g.manual_seed(N + d)
+    src = torch.randn((N, d), generator=g, device="cuda").to(torch.bfloat16)
+    out = handoff.receive_rows(src)
+    torch.cuda.synchronize()
+    assert np.array_equal(_bits(out), _bits(src))
+
+
+def test_valid_rows_only_and_fp32_rows():
+    import torch
+    from full_vocab_kl_b200 import handoff
+    x = make_custom(700, 128, 256, 1024, 1.0, 1.0, n_masked=200, teacher="independent", h_dtype="f32")
+    src = torch.from_numpy(x.h_t).cuda()
+    lab = torch.from_numpy(x.labels).cuda()
+    out = torch.full_like(src, 7.0)
+    handoff.receive_rows(src, lab, out=out)
+    torch.cuda.synchronize()
+    valid = x.labels != -100
+    assert np.array_equal(out.cpu().numpy()[valid], x.h_t[valid])
+    assert (out.cpu().numpy()[~valid] == 7.0).all()
+
+
+def test_zero_rows_and_argument_errors():
+    import torch
+    from full_vocab_kl_b200 import handoff
+    src = torch.zeros((0, 64), dtype=torch.bfloat16, device="cuda")
+    assert handoff.receive_rows(src).shape == (0, 64)
+    with pytest.raises(ValueError):
+        handoff.receive_rows(torch.zeros((4, 64), dtype=torch.bfloat16, device="cuda"),
+                             out=torch.zeros((4, 32), dtype=torch.bfloat16, device="cuda"))
+
+
+def _teacher(q, done, name):
+    import torch
+    from synthetic import make_inputs as mk
+    torch.cuda.set_device(0)
+    x = mk(name)
+    h_t = torch.from_numpy(x.h_t.view(np.int16)).cuda().view(torch.bfloat16)
+    torch.cuda.synchronize()
+    q.put(h_t)
+    done.wait(timeout=300)
+
+
+def _exclusive_compute_mode():
+    try:
+        r = subprocess.run(["nvidia-smi", "--query-gpu=compute_mode", "--format=csv,noheader", "-i", "0"],
+                           capture_output=True, text=True, timeout=30)
+        return "Exclusive" in r.stdout
+    except Exception:
+        return False
+
+
+def test_two_processes_through_ipc():
+    """The teacher process owns h_t; this process maps it, hands the valid rows over into local
+    memory and runs the loss on them — and on the mapped buffer directly. Both equal the loss on
+    a locally generated copy of the same bytes, bit for bit."""
+    if _exclusive_compute_mode():
+        pytest.skip("the GPU is in an exclusive compute mode: a second process cannot share it")
+    import torch
+    import torch.multiprocessing as mp
+    import full_vocab_kl_b200 as nb
+    from full_vocab_kl_b200 import handoff
+    name = "opd_0p6b_4b"
+    ctx = mp.get_context("spawn")
+    q, done = ctx.Queue(), ctx.Event()
+    p = ctx.Process(target=_teacher, args=(q, done, name))
+    p.start()
+    try:
+        remote = q.get(timeout=300)
+        x = make_inputs(name)
+        t = gu.torch_inputs(x)
+        local = handoff.receive_rows(remote, t["labels"])
+        torch.cuda.synchronize()
+        valid = x.labels != -100
+        assert np.array_equal(_bits(local)[valid], x.h_t.view(np.int16)[valid])
+        outs = []
+        for ht in (local, remote, t["h_t"]):
+            f = nb.kl_forward(t["h_s"], t["W_s"], ht, t["W_t"], t["labels"], x.beta, x.tau)
+            torch.cuda.synchronize()
+            outs.append({k: f[k].cpu().numpy() for k in ("loss_tok", "lse_t")})
+            assert nb.device_status(f["workspace"]) == 0
+        for o in outs[:2]:
+            for k in o:
+                assert np.array_equal(o[k], outs[2][k]), k
+        del remote
+    finally:
+        done.set()
+        p.join(timeout=120)
+        if p.is_alive():
+            p.kill()
+    assert p.exitcode == 0
