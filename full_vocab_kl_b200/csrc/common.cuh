@@ -117,9 +117,20 @@ struct GemmProb {
   int out_bf16;            // 1: out is bf16 (32 x 32 boxes, 64-byte swizzle), stored rounded to nearest even
 };
 
+// Wide GEMM tiles: 256 x 512 per CTA pair (two N = 256 accumulators, all of TMEM), 4 stages of
+// A 16 KB + B 2 x 16 KB per CTA. Each stage's operand bytes then feed twice the MMA work of
+// a 256 x 256 tile's stage with half again as many bytes: 25% fewer shared-memory writes
+// per FLOP.
+constexpr int kWideN = 2 * kBlockN;                         // 512
+constexpr int kWideStages = 4;
+constexpr int kWideStageBytes = kATileBytes + 2 * kBTileBytes;   // 48 KB per CTA
+constexpr int kWidePairStageBytes = 2 * kWideStageBytes;
+static_assert(kWideStages * kWideStageBytes == kStages * kStageBytes, "wide stages reuse the operand area");
+
 struct GemmArgs {
   GemmProb prob[2];
   int nprob;
+  int wide;                // 1: every tile is 256 x 512 (kWideN); 0: 256 x 256, double-buffered
   const int* n_valid;
   int* sched;              // zeroed work counter (null: static stride)
   int* status;

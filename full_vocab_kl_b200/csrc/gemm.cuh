@@ -28,32 +28,44 @@ __device__ __forceinline__ int prob_M(const GemmProb& q, int nv) { return q.m_dy
 __device__ __forceinline__ int prob_K(const GemmProb& q, int nv) {
   return q.k_dyn ? ((nv + kPairM - 1) / kPairM) * kPairM : q.K;
 }
-__device__ __forceinline__ int prob_tiles(const GemmProb& q, int nv) {
-  return ((prob_M(q, nv) + kPairM - 1) / kPairM) * ((q.N + kBlockN - 1) / kBlockN);
+__device__ __forceinline__ int prob_tiles(const GemmProb& q, int nv, int tile_n) {
+  return ((prob_M(q, nv) + kPairM - 1) / kPairM) * ((q.N + tile_n - 1) / tile_n);
 }
 
 __device__ __forceinline__ TileInfo tile_info(const GemmArgs& p, int nv, int tile) {
   TileInfo ti;
+  const int tile_n = p.wide ? kWideN : kBlockN;
   int pr = 0;
-  int t0 = prob_tiles(p.prob[0], nv);
+  int t0 = prob_tiles(p.prob[0], nv, tile_n);
   if (p.nprob > 1 && tile >= t0) {
     pr = 1;
     tile -= t0;
   }
   const GemmProb& q = p.prob[pr];
-  const int n_tiles = (q.N + kBlockN - 1) / kBlockN;
+  const int n_tiles = (q.N + tile_n - 1) / tile_n;
   ti.prob = pr;
   ti.m0 = (tile / n_tiles) * kPairM;
-  ti.n0 = (tile % n_tiles) * kBlockN;
+  ti.n0 = (tile % n_tiles) * tile_n;
   ti.nkb = (prob_K(q, nv) + kBlockK - 1) / kBlockK;
   ti.M = prob_M(q, nv);
   return ti;
 }
 
 __device__ __forceinline__ int total_tiles(const GemmArgs& p, int nv) {
-  int t = prob_tiles(p.prob[0], nv);
-  if (p.nprob > 1) t += prob_tiles(p.prob[1], nv);
+  const int tile_n = p.wide ? kWideN : kBlockN;
+  int t = prob_tiles(p.prob[0], nv, tile_n);
+  if (p.nprob > 1) t += prob_tiles(p.prob[1], nv, tile_n);
   return t;
+}
+
+// Shared-memory addresses of stage `st`'s operands: narrow tiles keep A and B in two arrays
+// of kStages x 16 KB; wide tiles use the same 192 KB as kWideStages x (A, B half 0, B half 1).
+__device__ __forceinline__ uint32_t stage_a(const SweepSmem& s, int wide, int st) {
+  return wide ? smem_addr(s.a + st * kWideStageBytes) : smem_addr(s.a + st * kATileBytes);
+}
+__device__ __forceinline__ uint32_t stage_b(const SweepSmem& s, int wide, int st, int half) {
+  return wide ? smem_addr(s.a + st * kWideStageBytes + kATileBytes + half * kBTileBytes)
+              : smem_addr(s.b + st * kBTileBytes);
 }
 
 // K-major operand: one (rows x 64) box. MN-major operand: (rows / 64) boxes of 64 x 64
@@ -83,6 +95,7 @@ __device__ __forceinline__ void gemm_producer(const GemmMaps& maps, const GemmAr
   int n_issued = 0;
   bool ok = true;
   const int nt = total_tiles(p, nv);
+  const int n_stages = p.wide ? kWideStages : kStages;
   for (int it = 0; ok; ++it) {
     int tile;
     if (rank == 0) {
@@ -100,18 +113,20 @@ __device__ __forceinline__ void gemm_producer(const GemmMaps& maps, const GemmAr
     for (int kb = 0; kb < ti.nkb; ++kb) {
       if (!mbar_wait_cl(&s.empty[stage], phase ^ 1u, w)) { ok = false; break; }
       const uint32_t bar = smem_addr(&s.full[stage]);
-      if (rank == 0) mbar_arrive_expect_tx(&s.full[stage], kPairStageBytes);
-      load_operand(smem_addr(s.a + stage * kATileBytes), &maps.a[ti.prob], bar, q.a_mn, am0,
-                   q.a_koff + kb * kBlockK, kBlockM);
-      load_operand(smem_addr(s.b + stage * kBTileBytes), &maps.b[ti.prob], bar, q.b_mn, bn0,
-                   q.b_koff + kb * kBlockK, kHalfB);
+      if (rank == 0) mbar_arrive_expect_tx(&s.full[stage], p.wide ? kWidePairStageBytes : kPairStageBytes);
+      const int kc = kb * kBlockK;
+      load_operand(stage_a(s, p.wide, stage), &maps.a[ti.prob], bar, q.a_mn, am0, q.a_koff + kc, kBlockM);
+      load_operand(stage_b(s, p.wide, stage, 0), &maps.b[ti.prob], bar, q.b_mn, bn0, q.b_koff + kc, kHalfB);
+      if (p.wide)   // the second 256-column half of the tile: this CTA's 128 of its B rows
+        load_operand(stage_b(s, 1, stage, 1), &maps.b[ti.prob], bar, q.b_mn, bn0 + kBlockN, q.b_koff + kc,
+                     kHalfB);
       pend_stage[n_issued % kStages] = stage;
       pend_par[n_issued % kStages] = phase;
       ++n_issued;
-      if (++stage == kStages) { stage = 0; phase ^= 1u; }
+      if (++stage == n_stages) { stage = 0; phase ^= 1u; }
     }
   }
-  if (!ok && rank == 0) drain_loads(s, pend_stage, pend_par, n_issued);
+  if (!ok && rank == 0) drain_loads(s, pend_stage, pend_par, n_issued, n_stages);
 }
 
 __device__ __forceinline__ void gemm_mma(const GemmArgs& p, int nv, const SweepSmem& s, uint32_t tmem_base,
@@ -128,14 +143,43 @@ __device__ __forceinline__ void gemm_mma(const GemmArgs& p, int nv, const SweepS
     const TileInfo ti = tile_info(p, nv, tile);
     const GemmProb& q = p.prob[ti.prob];
     const uint32_t idesc = make_idesc(kPairM, kBlockN, q.a_mn, q.b_mn);
+    if (p.wide) {
+      // both accumulators hold this tile: columns [n0, n0 + 256) in buffer 0, the next 256 in 1
+      if (!mbar_wait_cl(&s.tempty[0], acc_phase ^ 1u, w) || !mbar_wait_cl(&s.tempty[1], acc_phase ^ 1u, w)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      for (int kb = 0; kb < ti.nkb; ++kb) {
+        if (!mbar_wait(&s.full[stage], phase, w)) { ok = false; break; }
+        const uint32_t sa = stage_a(s, 1, stage);
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const uint32_t sb = stage_b(s, 1, stage, h);
+#pragma unroll
+          for (int j = 0; j < kBlockK / 16; ++j)
+            umma_bf16_pair(tmem_base + h * kBlockN, operand_desc(sa, q.a_mn, j), operand_desc(sb, q.b_mn, j),
+                           idesc, (kb > 0 || j > 0) ? 1u : 0u);
+          // the first half is complete one half-step early: its epilogue starts meanwhile
+          if (h == 0 && kb == ti.nkb - 1) umma_commit_pair_both(smem_addr(&s.tfull[0]));
+        }
+        umma_commit_pair_both(smem_addr(&s.empty[stage]));
+        if (++stage == kWideStages) { stage = 0; phase ^= 1u; }
+      }
+      if (!ok) break;
+      if (ti.nkb == 0) umma_commit_pair_both(smem_addr(&s.tfull[0]));
+      umma_commit_pair_both(smem_addr(&s.tfull[1]));
+      acc_phase ^= 1u;
+      continue;
+    }
     if (!mbar_wait_cl(&s.tempty[acc], acc_phase ^ 1u, w)) { ok = false; break; }
     tc_fence_after();
     const uint32_t d = tmem_base + acc * kBlockN;
     for (int kb = 0; kb < ti.nkb; ++kb) {
       // TMA bytes are ordered by the barrier's transaction count: no tcgen05 fence here
       if (!mbar_wait(&s.full[stage], phase, w)) { ok = false; break; }
-      const uint32_t sa = smem_addr(s.a + stage * kATileBytes);
-      const uint32_t sb = smem_addr(s.b + stage * kBTileBytes);
+      const uint32_t sa = stage_a(s, 0, stage);
+      const uint32_t sb = stage_b(s, 0, stage, 0);
 #pragma unroll
       for (int j = 0; j < kBlockK / 16; ++j) {
         umma_bf16_pair(d, operand_desc(sa, q.a_mn, j), operand_desc(sb, q.b_mn, j), idesc,
@@ -177,6 +221,10 @@ __device__ __forceinline__ void gemm_epilogue(const GemmMaps& maps, const GemmAr
     const TileInfo ti = tile_info(p, nv, tile);
     const GemmProb& q = p.prob[ti.prob];
     const int row0 = ti.m0 + int(rank) * kBlockM + qq * 32;   // first of the warp's 32 rows
+    // a wide tile is read as two 256-column tiles, from accumulator buffers 0 and 1 in turn
+#pragma unroll 1
+    for (int sub = 0; sub < (p.wide ? 2 : 1); ++sub) {
+    const int n0 = ti.n0 + sub * kBlockN;
     if (!mbar_wait_cl(&s.tfull[acc], acc_phase, w)) return;
     tc_fence_after();
     const uint32_t base = tmem_base + lane_addr + acc * kBlockN + half * kHalfN;
@@ -190,7 +238,7 @@ __device__ __forceinline__ void gemm_epilogue(const GemmMaps& maps, const GemmAr
 #pragma unroll
         for (int j = 0; j < 32; ++j) v[j] = 0.f;
       }
-      const int c0 = ti.n0 + half * kHalfN + ch * 32;
+      const int c0 = n0 + half * kHalfN + ch * 32;
       if (c0 >= q.N || row0 >= ti.M) continue;
       if (staged && lane == 0) bulk_wait_read();
       __syncwarp();
@@ -222,6 +270,7 @@ __device__ __forceinline__ void gemm_epilogue(const GemmMaps& maps, const GemmAr
     }
     acc ^= 1;
     if (acc == 0) acc_phase ^= 1u;
+    }
   }
   if (lane == 0) bulk_wait_all();
 }

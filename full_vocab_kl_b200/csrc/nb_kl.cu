@@ -366,6 +366,11 @@ unsigned pair_grid(const DevInfo& dev, int work_items) {
   return unsigned(2 * std::max(1, std::min(dev.pairs, work_items)));
 }
 
+// Wide (256 x 512) GEMM tiles when they cover the N columns with no more padding than
+// 256-wide tiles; their output column tile width.
+int gemm_wide(int64_t N) { return round_up(N, 2 * kBlockN) == round_up(N, kBlockN) ? 1 : 0; }
+int gemm_tile_n(int wide) { return wide ? kWideN : kBlockN; }
+
 int sweep_units(const Layout& L, const SweepArgs& a) {
   const int n_tt = int(L.N_pad / kPairM);
   const int n_vt = (a.v_end - a.v_begin + kBlockN - 1) / kBlockN;
@@ -781,6 +786,7 @@ nb_status nb_kl_backward(const nb_kl_shape* shape, const void* h_s, const void* 
   GemmArgs g;
   std::memset(&g, 0, sizeof(g));
   g.nprob = 2;
+  g.wide = gemm_wide(L.d_s);
   g.n_valid = &w.ctrl->n_valid;
   g.status = &w.ctrl->status;
   g.wait_limit_ns = kWaitLimitNs;
@@ -798,7 +804,7 @@ nb_status nb_kl_backward(const nb_kl_shape* shape, const void* h_s, const void* 
   dw.accumulate = accumulate_dW ? 1 : 0;
 
   const int n_tt_max = int(L.N_pad / kPairM);
-  const int n_dt = int((L.d_s + kBlockN - 1) / kBlockN);   // 256-wide output column tiles
+  const int n_dt = int((L.d_s + gemm_tile_n(g.wide) - 1) / gemm_tile_n(g.wide));   // output column tiles
   AuxStream* ax = nullptr;
   if ((s = aux_stream(&ax)) != NB_OK) return s;
   // fork: the GEMMs run on a second stream, ordered after everything before this call
@@ -887,7 +893,8 @@ nb_status nb_kl_gram(const void* X, int64_t rows, int64_t d, float* G, void* wor
   q.M = int(d);
   q.N = int(d);
   q.K = int(rows);
-  const int tiles = int((d + kPairM - 1) / kPairM * ((d + kBlockN - 1) / kBlockN));
+  g.wide = gemm_wide(d);
+  const int tiles = int((d + kPairM - 1) / kPairM * ((d + gemm_tile_n(g.wide) - 1) / gemm_tile_n(g.wide)));
   next_cat(NB_KL_KERNEL_GEMM_PROJ);
   launch(gemm_kernel, dim3(pair_grid(dev, tiles)), dim3(kThreads), size_t(kSmemBytes), st, gm, g);
   return check_launch();
@@ -927,7 +934,8 @@ nb_status nb_kl_project(const void* X, int64_t rows, int64_t d, const void* B, i
   q.N = int(k);
   q.K = int(d);
   q.out_bf16 = 1;
-  const int tiles = int((rows + kPairM - 1) / kPairM * ((k + kBlockN - 1) / kBlockN));
+  g.wide = gemm_wide(k);
+  const int tiles = int((rows + kPairM - 1) / kPairM * ((k + gemm_tile_n(g.wide) - 1) / gemm_tile_n(g.wide)));
   next_cat(NB_KL_KERNEL_GEMM_PROJ);
   launch(gemm_kernel, dim3(pair_grid(dev, tiles)), dim3(kThreads), size_t(kSmemBytes), st, gm, g);
   return check_launch();
@@ -1001,7 +1009,8 @@ nb_status nb_kl_debug_gemm(const void* A, int a_mn_major, const void* B, int b_m
   q.K = int(K);
   ok = make_out_map(&gm.out[0], C, N, M);
   if (!ok) return NB_ERR_CUDA;
-  const int tiles = int((M + kPairM - 1) / kPairM * ((N + kBlockN - 1) / kBlockN));
+  g.wide = gemm_wide(N);
+  const int tiles = int((M + kPairM - 1) / kPairM * ((N + gemm_tile_n(g.wide) - 1) / gemm_tile_n(g.wide)));
   launch(gemm_kernel, dim3(pair_grid(dev, tiles)), dim3(kThreads), size_t(kSmemBytes), st, gm, g);
   return check_launch();
 }

@@ -307,4 +307,39 @@ __device__ __forceinline__ float lg2(float x) {
   return y;
 }
 
+// ------------------------------------------------------------------ packed fp32 pairs
+// Two fp32 lanes in one 64-bit register: one f32x2 instruction does the work of two scalar
+// ones on the FMA pipe (round to nearest even, like the scalar forms).
+struct f2 {
+  uint64_t v;
+};
+__device__ __forceinline__ f2 pk2(float lo, float hi) {
+  f2 r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r.v) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void upk2(f2 a, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(a.v));
+}
+__device__ __forceinline__ f2 fma2(f2 a, f2 b, f2 c) {
+  f2 d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d.v) : "l"(a.v), "l"(b.v), "l"(c.v));
+  return d;
+}
+__device__ __forceinline__ f2 mul2(f2 a, f2 b) {
+  f2 d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d.v) : "l"(a.v), "l"(b.v));
+  return d;
+}
+__device__ __forceinline__ f2 add2(f2 a, f2 b) {
+  f2 d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d.v) : "l"(a.v), "l"(b.v));
+  return d;
+}
+__device__ __forceinline__ float sum2(f2 a) {
+  float lo, hi;
+  upk2(a, lo, hi);
+  return lo + hi;
+}
+
 }  // namespace nbkl

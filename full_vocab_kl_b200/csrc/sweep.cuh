@@ -167,8 +167,8 @@ __device__ __forceinline__ bool ring_get(const SweepSmem& s, int it, int& id, co
 // Bounded wait for the copies a failed producer may still have in flight (leader: its full[]
 // barriers count the bytes of both CTAs).
 __device__ __forceinline__ void drain_loads(const SweepSmem& s, const uint32_t* pend_stage,
-                                            const uint32_t* pend_par, int n_issued) {
-  const int n = min(n_issued, kStages);
+                                            const uint32_t* pend_par, int n_issued, int n_stages = kStages) {
+  const int n = min(n_issued, n_stages);
   for (int i = 0; i < n; ++i) {
     const int j = (n_issued - 1 - i) % kStages;
     const uint32_t a = smem_addr(&s.full[pend_stage[j]]);
@@ -299,20 +299,25 @@ struct RowState {
   float ms, ls, mt, lt, a, e;
 };
 
+// One 32-column chunk of a row: zs / zt hold the raw logits z. The maxima are taken on z (the
+// scale log2(e) / tau is positive) and every exponent is formed as fma(z, scale, -m), so the
+// scaled logits are never stored; the KL numerator sums 2^(x - m) (z_s - z_t) in raw units and
+// is scaled once per chunk. Column pairs go through the packed f32x2 forms.
 template <int MODE, bool MASKED, bool SIDE>
 __device__ __forceinline__ void chunk_state(float (&zs)[32], float (&zt)[32], int n_ok, float scale, RowState& r,
                                             int lab_off, float* lab_dst) {
-  float cs = kNegBig, ct = kNegBig;
+  if (MASKED) {
 #pragma unroll
-  for (int j = 0; j < 32; ++j) {
-    float xs = zs[j] * scale, xt = zt[j] * scale;
-    if (MASKED && j >= n_ok) { xs = kNegBig; xt = kNegBig; }
-    zs[j] = xs;
-    zt[j] = xt;
-    cs = fmaxf(cs, xs);
-    ct = fmaxf(ct, xt);
+    for (int j = 0; j < 32; ++j)
+      if (j >= n_ok) { zs[j] = kNegBig; zt[j] = kNegBig; }
   }
-  const float ns = fmaxf(r.ms, cs), nt = fmaxf(r.mt, ct);
+  float cs = zs[0], ct = zt[0];
+#pragma unroll
+  for (int j = 1; j < 32; ++j) {
+    cs = fmaxf(cs, zs[j]);
+    ct = fmaxf(ct, zt[j]);
+  }
+  const float ns = fmaxf(r.ms, cs * scale), nt = fmaxf(r.mt, ct * scale);
   const float rs = ex2(r.ms - ns), rt = ex2(r.mt - nt);
   // re-centre e on the new maximum: sum 2^(x - ns) (x - ns) = rs (e + (ms - ns) l)
   if (SIDE) r.e = rs * fmaf(r.ms - ns, r.ls, r.e);
@@ -322,29 +327,41 @@ __device__ __forceinline__ void chunk_state(float (&zs)[32], float (&zt)[32], in
   if (MODE == kStateT) r.a *= rt;
   r.ms = ns;
   r.mt = nt;
-  float ls = 0.f, lt = 0.f, a = 0.f, e = 0.f;
+  const f2 sc = pk2(scale, scale), mns = pk2(-ns, -ns), mnt = pk2(-nt, -nt), m1 = pk2(-1.f, -1.f);
+  f2 ls = pk2(0.f, 0.f), lt = ls, a = ls, e = ls;
 #pragma unroll
-  for (int j = 0; j < 32; ++j) {
-    const float ds = zs[j] - ns;
-    const float es = ex2(ds);
-    const float et = ex2(zt[j] - nt);
-    ls += es;
-    lt += et;
-    if (SIDE) e = fmaf(es, ds, e);
-    if (MODE == kStateS) a = fmaf(es, zs[j] - zt[j], a);
-    if (MODE == kStateT) a = fmaf(et, zt[j] - zs[j], a);
+  for (int j = 0; j < 32; j += 2) {
+    const f2 z_s = pk2(zs[j], zs[j + 1]), z_t = pk2(zt[j], zt[j + 1]);
+    f2 ds = fma2(z_s, sc, mns), dt = fma2(z_t, sc, mnt);   // x - m
+    float d0, d1, t0, t1;
+    upk2(ds, d0, d1);
+    upk2(dt, t0, t1);
+    if (MASKED) {
+      // columns past the vocabulary contribute exactly 0 whatever the running maximum (when a
+      // thread's first chunk is all masked, fma(z, scale, -m) would leave the product's
+      // rounding error of a huge value here instead of 0)
+      if (j >= n_ok) d0 = t0 = kNegBig;
+      if (j + 1 >= n_ok) d1 = t1 = kNegBig;
+      ds = pk2(d0, d1);
+    }
+    const f2 es = pk2(ex2(d0), ex2(d1)), et = pk2(ex2(t0), ex2(t1));
+    ls = add2(ls, es);
+    lt = add2(lt, et);
+    if (SIDE) e = fma2(es, ds, e);
+    if (MODE == kStateS) a = fma2(es, fma2(z_t, m1, z_s), a);
+    if (MODE == kStateT) a = fma2(et, fma2(z_s, m1, z_t), a);
   }
-  r.ls += ls;
-  r.lt += lt;
-  r.a += a;
+  r.ls += sum2(ls);
+  r.lt += sum2(lt);
+  if (MODE == kStateS || MODE == kStateT) r.a = fmaf(sum2(a), scale, r.a);
   if (SIDE) {
-    r.e += e;
+    r.e += sum2(e);
     // the one thread whose chunk holds the row's label keeps that logit (a rare branch)
     if (unsigned(lab_off) < 32u) {
-      float x = 0.f;
+      float z = 0.f;
 #pragma unroll
-      for (int j = 0; j < 32; ++j) x = (j == lab_off) ? zs[j] : x;
-      *lab_dst = x;
+      for (int j = 0; j < 32; ++j) z = (j == lab_off) ? zs[j] : z;
+      *lab_dst = z * scale;
     }
   }
 }
@@ -399,10 +416,29 @@ template <int MODE, bool MASKED>
 __device__ __forceinline__ void chunk_grad(const float (&zs)[32], const float (&zt)[32], int n_ok, float scale,
                                            const RowConst& c, float gs, uint8_t* stage_row, int r) {
   uint32_t packed[16];
+  // the two KL directions in packed pairs: y = fma(z, scale, -L2) are the base-2 log-probabilities
+  const f2 sc = pk2(scale, scale), ms = pk2(-c.l2s, -c.l2s), mt = pk2(-c.l2t, -c.l2t), m1 = pk2(-1.f, -1.f);
+  const f2 ln2 = pk2(kLn2, kLn2), maux = pk2(-c.aux, -c.aux), g2 = pk2(gs, gs);
 #pragma unroll
   for (int j = 0; j < 32; j += 2) {
-    float g0 = gs * grad_elem<MODE>(zs[j] * scale, zt[j] * scale, c);
-    float g1 = gs * grad_elem<MODE>(zs[j + 1] * scale, zt[j + 1] * scale, c);
+    float g0, g1;
+    if (MODE == kGradFkl || MODE == kGradRkl) {
+      const f2 ys = fma2(pk2(zs[j], zs[j + 1]), sc, ms), yt = fma2(pk2(zt[j], zt[j + 1]), sc, mt);
+      float s0, s1, t0, t1;
+      upk2(ys, s0, s1);
+      upk2(yt, t0, t1);
+      const f2 S = pk2(ex2(s0), ex2(s1));
+      f2 g;
+      if (MODE == kGradFkl) {
+        g = fma2(pk2(ex2(t0), ex2(t1)), m1, S);                    // S - T
+      } else {
+        g = mul2(S, fma2(ln2, fma2(yt, m1, ys), maux));            // S (ln S - ln T - KL)
+      }
+      upk2(mul2(g, g2), g0, g1);
+    } else {
+      g0 = gs * grad_elem<MODE>(zs[j] * scale, zt[j] * scale, c);
+      g1 = gs * grad_elem<MODE>(zs[j + 1] * scale, zt[j + 1] * scale, c);
+    }
     if (MASKED && j >= n_ok) g0 = 0.f;
     if (MASKED && j + 1 >= n_ok) g1 = 0.f;
     __nv_bfloat162 h = __floats2bfloat162_rn(g0, g1);

@@ -73,7 +73,7 @@ def check_forward(got, ref, labels, rows=None):
     sel = np.flatnonzero(valid) if rows is None else np.asarray([r for r in rows if valid[r]])
     assert got["n_valid"] == int(valid.sum())
     lt, rt = got["loss_tok"][sel], ref["loss_tok"][sel]
-    bad = np.abs(lt - rt) > TOL_TOK_REL * np.abs(rt) + TOL_TOK_ABS
+    bad = ~(np.abs(lt - rt) <= TOL_TOK_REL * np.abs(rt) + TOL_TOK_ABS)   # NaN counts as off
     assert not bad.any(), f"per-token loss: {bad.sum()} rows off, worst {np.abs(lt - rt)[bad].max()}"
     for k in ("lse_s", "lse_t"):
         err = np.abs(got[k][sel] - ref[k][sel]) / np.maximum(np.abs(ref[k][sel]), 1e-30)
@@ -89,6 +89,7 @@ def check_forward(got, ref, labels, rows=None):
             assert got["loss_mean"] == 0.0
         else:
             assert abs(got["loss_mean"] - m) <= TOL_MEAN * abs(m) + 1e-7, (got["loss_mean"], m)
+    assert np.isfinite(got["loss_tok"]).all() and np.isfinite(got["loss_mean"])
 
 
 def check_side(got, ref, labels, V, rows=None):

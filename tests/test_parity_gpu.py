@@ -136,3 +136,12 @@ def test_repeatable():
     for k in ("loss_tok", "lse_s", "aux", "dh_s", "dW_s"):
         np.testing.assert_array_equal(a[k], b[k])
     assert a["loss_mean"] == b["loss_mean"]
+
+
+@pytest.mark.parametrize("V", [100, 2148, 4224])
+@pytest.mark.parametrize("beta", [0.0, 1.0, 0.5])
+def test_vocab_tail_leaves_whole_column_halves_empty(V, beta):
+    # V mod 2048 <= 128 (or V <= 128): the last work unit's only tile has a column half that
+    # lies entirely past the vocabulary, so some epilogue threads start on an all-masked chunk
+    x = make_custom(300, 128, 192, V, beta, 0.7, n_masked=40, teacher="correlated")
+    full_check(x)

@@ -137,3 +137,9 @@ def test_full_size_sampled_rows(name):
     H = got["entropy_s"][valid]
     assert (H >= -1e-5).all() and (H <= np.log(x.W_s.shape[0]) + 1e-4).all()
     assert (got["logp_label"][valid] <= 1e-5).all()
+
+
+@pytest.mark.parametrize("V", [100, 2148])
+def test_side_outputs_with_empty_column_halves(V):
+    x = make_custom(300, 128, 192, V, 0.5, 0.7, n_masked=40, teacher="correlated")
+    check(x)
