@@ -79,7 +79,7 @@ struct SweepArgs {
   int bmod_s, bmod_t;     // B block of A block kb is kb % bmod (fp32 hi/lo split reuses W)
   int tiles_per_unit;     // vocabulary tiles per work unit (one split of the LSE state)
   float scale;            // log2(e) / tau: base-2 tempered logits x = z * scale
-  float beta, lg2_1mb, lg2_b;
+  float beta;
   float* out;             // state [6][split][ld] or JSD partial sums [2][split][ld]; split =
                           // 2 * unit + column half
   long long field_stride; // elements between fields of `out`

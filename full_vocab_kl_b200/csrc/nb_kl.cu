@@ -347,8 +347,6 @@ SweepArgs base_sweep_args(const Layout& L, const Ws& w, float beta, float tau) {
   a.tiles_per_unit = kTilesPerUnitFwd;
   a.scale = float(1.4426950408889634 / double(tau));
   a.beta = beta;
-  a.lg2_1mb = (beta < 1.f) ? float(std::log2(1.0 - double(beta))) : 0.f;
-  a.lg2_b = (beta > 0.f) ? float(std::log2(double(beta))) : 0.f;
   a.ld = int(L.N_pad);
   a.field_stride = L.fs_state;
   a.row_l2s = w.rl2s;

@@ -368,45 +368,43 @@ __device__ __forceinline__ void chunk_state(float (&zs)[32], float (&zt)[32], in
 
 struct RowConst {
   float l2s, l2t, aux;
-  float beta, omb, lg2_1mb, lg2_b;
+  float beta, omb;
 };
 
-// log2 of the mixture M = (1 - beta) S + beta T from base-2 log-probabilities.
-__device__ __forceinline__ float log2_mixture(float ys, float yt, const RowConst& c) {
-  const float a = ys + c.lg2_1mb, b = yt + c.lg2_b;
-  const float hi = fmaxf(a, b), lo = fminf(a, b);
-  return hi + lg2(1.0f + ex2(lo - hi));
+// log2 of the mixture M = (1 - beta) S + beta T from S and T themselves, floored at 2^-126:
+// where both have underflowed every term that uses it is below 2^-126 anyway.
+__device__ __forceinline__ f2 log2_mix2(f2 S, f2 T, f2 omb, f2 bb) {
+  float m0, m1;
+  upk2(fma2(bb, T, mul2(omb, S)), m0, m1);
+  return pk2(lg2(fmaxf(m0, 0x1p-126f)), lg2(fmaxf(m1, 0x1p-126f)));
 }
 
+// JSD pass: js += beta sum T (y_t - y_m) + (1 - beta) sum S (y_s - y_m), ks += sum S (y_s - y_m)
+// (base 2, converted to nats by the finalisation), column pairs in packed form.
 template <bool MASKED>
 __device__ __forceinline__ void chunk_jsd(const float (&zs)[32], const float (&zt)[32], int n_ok, float scale,
                                           const RowConst& c, float& js, float& ks) {
-  float j_acc = 0.f, k_acc = 0.f;
+  const f2 sc = pk2(scale, scale), ms = pk2(-c.l2s, -c.l2s), mt = pk2(-c.l2t, -c.l2t), m1 = pk2(-1.f, -1.f);
+  const f2 omb = pk2(c.omb, c.omb), bb = pk2(c.beta, c.beta);
+  f2 k_acc = pk2(0.f, 0.f), j_acc = k_acc;
 #pragma unroll
-  for (int j = 0; j < 32; ++j) {
-    const float ys = fmaf(zs[j], scale, -c.l2s);
-    const float yt = fmaf(zt[j], scale, -c.l2t);
-    float S = ex2(ys), T = ex2(yt);
-    if (MASKED && j >= n_ok) { S = 0.f; T = 0.f; }
-    const float ym = log2_mixture(ys, yt, c);
-    const float ds = ys - ym, dt = yt - ym;
-    k_acc = fmaf(S, ds, k_acc);
-    j_acc = fmaf(c.beta * T, dt, j_acc);
+  for (int j = 0; j < 32; j += 2) {
+    const f2 ys = fma2(pk2(zs[j], zs[j + 1]), sc, ms), yt = fma2(pk2(zt[j], zt[j + 1]), sc, mt);
+    float s0, s1, t0, t1;
+    upk2(ys, s0, s1);
+    upk2(yt, t0, t1);
+    float S0 = ex2(s0), S1 = ex2(s1), T0 = ex2(t0), T1 = ex2(t1);
+    if (MASKED && j >= n_ok) S0 = T0 = 0.f;
+    if (MASKED && j + 1 >= n_ok) S1 = T1 = 0.f;
+    const f2 S = pk2(S0, S1), T = pk2(T0, T1);
+    const f2 ym = log2_mix2(S, T, omb, bb);
+    k_acc = fma2(S, fma2(ym, m1, ys), k_acc);
+    j_acc = fma2(T, fma2(ym, m1, yt), j_acc);
   }
   // JSD = beta * KL(T||M) + (1 - beta) * KL(S||M); the S term is the K accumulator
-  js += j_acc + c.omb * k_acc;
-  ks += k_acc;
-}
-
-// d loss_n / d u_s for one element, base-2 inputs.
-template <int MODE>
-__device__ __forceinline__ float grad_elem(float xs, float xt, const RowConst& c) {
-  const float ys = xs - c.l2s, yt = xt - c.l2t;
-  const float S = ex2(ys);
-  if (MODE == kGradFkl) return S - ex2(yt);
-  if (MODE == kGradRkl) return S * fmaf(kLn2, ys - yt, -c.aux);
-  const float ym = log2_mixture(ys, yt, c);
-  return c.omb * S * fmaf(kLn2, ys - ym, -c.aux);
+  const float k = sum2(k_acc);
+  js += fmaf(c.beta, sum2(j_acc), c.omb * k);
+  ks += k;
 }
 
 // Gradient of one 32-column chunk of a row, packed to bf16 and written into the warp's
@@ -436,8 +434,15 @@ __device__ __forceinline__ void chunk_grad(const float (&zs)[32], const float (&
       }
       upk2(mul2(g, g2), g0, g1);
     } else {
-      g0 = gs * grad_elem<MODE>(zs[j] * scale, zt[j] * scale, c);
-      g1 = gs * grad_elem<MODE>(zs[j + 1] * scale, zt[j + 1] * scale, c);
+      // (1 - beta) S (ln S - ln M - K)
+      const f2 ys = fma2(pk2(zs[j], zs[j + 1]), sc, ms), yt = fma2(pk2(zt[j], zt[j + 1]), sc, mt);
+      float s0, s1, t0, t1;
+      upk2(ys, s0, s1);
+      upk2(yt, t0, t1);
+      const f2 S = pk2(ex2(s0), ex2(s1)), T = pk2(ex2(t0), ex2(t1));
+      const f2 ym = log2_mix2(S, T, pk2(c.omb, c.omb), pk2(c.beta, c.beta));
+      const f2 g = mul2(mul2(S, pk2(c.omb, c.omb)), fma2(ln2, fma2(ym, m1, ys), maux));
+      upk2(mul2(g, g2), g0, g1);
     }
     if (MASKED && j >= n_ok) g0 = 0.f;
     if (MASKED && j + 1 >= n_ok) g1 = 0.f;
@@ -491,8 +496,6 @@ __device__ __forceinline__ void sweep_epilogue(const SweepMaps& maps, const Swee
   RowConst c;
   c.beta = p.beta;
   c.omb = 1.0f - p.beta;
-  c.lg2_1mb = p.lg2_1mb;
-  c.lg2_b = p.lg2_b;
   const float gscale = (MODE >= kGradFkl) ? *p.gscale : 0.f;
 
   for (int it = 0;; ++it) {
