@@ -27,7 +27,7 @@ def input_hashes(x):
 
 def main():
     x = make_inputs("tiny", seed=0)
-    f = oracle.forward(x.h_s, x.W_s, x.h_t, x.W_t, x.labels, x.beta, x.tau)
+    f = oracle.forward(x.h_s, x.W_s, x.h_t, x.W_t, x.labels, x.beta, x.tau, side=True)
     b = oracle.backward(x.h_s, x.W_s, x.h_t, x.W_t, x.labels, x.beta, x.tau)
     out = {
         "source": "tests/golden/make_golden.py (oracle only), workload 'tiny', seed 0",
@@ -37,6 +37,8 @@ def main():
         "loss_tok_first8_valid": [float(v) for v in f["loss_tok"][32:40]],
         "lse_s_first8_valid": [float(v) for v in f["lse_s"][32:40]],
         "lse_t_first8_valid": [float(v) for v in f["lse_t"][32:40]],
+        "entropy_s_first8_valid": [float(v) for v in f["entropy_s"][32:40]],
+        "logp_label_first8_valid": [float(v) for v in f["logp_label"][32:40]],
         "dh_s_fro": float(np.linalg.norm(b["dh_s"])),
         "dW_s_fro": float(np.linalg.norm(b["dW_s"])),
     }

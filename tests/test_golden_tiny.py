@@ -22,8 +22,10 @@ def test_tiny_golden():
         g = json.load(f)
     x = make_inputs("tiny", seed=0)
     assert mg.input_hashes(x) == g["hashes"]
-    fw = oracle.forward(x.h_s, x.W_s, x.h_t, x.W_t, x.labels, x.beta, x.tau)
+    fw = oracle.forward(x.h_s, x.W_s, x.h_t, x.W_t, x.labels, x.beta, x.tau, side=True)
     assert fw["n_valid"] == g["n_valid"] == 96
+    np.testing.assert_allclose(fw["entropy_s"][32:40], g["entropy_s_first8_valid"], rtol=1e-12)
+    np.testing.assert_allclose(fw["logp_label"][32:40], g["logp_label_first8_valid"], rtol=1e-12)
     assert fw["loss_mean"] == pytest.approx(g["loss_mean"], rel=1e-12)
     np.testing.assert_allclose(fw["loss_tok"][32:40], g["loss_tok_first8_valid"], rtol=1e-12)
     np.testing.assert_allclose(fw["lse_s"][32:40], g["lse_s_first8_valid"], rtol=1e-13)
