@@ -438,7 +438,7 @@ def run_library(args):
     copy_stream = torch.cuda.Stream(dev)
     h2d = sum(t.numel() * t.element_size() for t in pin.values())
     d2h = out["loss_mean"].element_size() + out["n_valid"].element_size()
-    e2e_steps = max(3, min(args.steps, 20))
+    e2e_steps = max(3, args.steps)   # as many steps as the device-timed region
 
     def issue_copy(i):
         # buffer i % 2 was last read by step i - 2, which the host has already waited for
