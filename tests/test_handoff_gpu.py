@@ -2,9 +2,9 @@
 4/8: the teacher's final hidden state crosses to the loss instead of V logits per token).
 
 A byte copy: results must be bit-exact. The two-process test shares the teacher's buffer
-through CUDA IPC (a CUDA tensor sent through a torch.multiprocessing queue); every gpurun call
-has one GPU, so both processes use it: the transfer is then an HBM copy, the code path (an IPC
-mapping read by plain loads) is the one a second GPU would use over NVLink. The processes do
+through CUDA IPC (a CUDA tensor sent through a torch.multiprocessing queue); both processes use
+GPU 0, so the transfer is an HBM copy, while the code path (an IPC mapping read by plain loads)
+is the one a second GPU would use over NVLink. The processes do
 not wait on each other inside kernels: the hand-over is a host queue and a host event, both
 with timeouts.
 """
