@@ -48,3 +48,25 @@ def test_reference_arm_runs_on_rank0_only(monkeypatch, capsys):
     args = argparse.Namespace(workload="tiny", steps=3, warmup=3)
     assert bench.run_reference(args) == 0
     assert capsys.readouterr().out == ""
+
+
+def test_reference_arm_line_on_rank0(monkeypatch, capsys):
+    """The reference arm (the oracle on the host cores) prints one JSON line with the keys the
+    benchmark contract asks for."""
+    import argparse
+    import json
+    import bench
+    monkeypatch.setenv("RANK", "0")
+    monkeypatch.setenv("WORLD_SIZE", "1")
+    args = argparse.Namespace(workload="tiny", steps=3, warmup=3)
+    assert bench.run_reference(args) == 0
+    lines = [l for l in capsys.readouterr().out.splitlines() if l.strip()]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["unit"] == "tokens/s" and d["value"] > 0
+    assert d["metric"] == bench.METRIC and d["higher_is_better"] is True
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
+    assert d["cpu_baseline"]["value"] == d["value"] and d["cpu_baseline"]["sample"]
+    assert d["e2e"] == {"value": d["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}
+    assert d["config"]["workload"] == "tiny"
