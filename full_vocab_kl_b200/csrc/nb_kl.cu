@@ -365,8 +365,12 @@ unsigned pair_grid(const DevInfo& dev, int work_items) {
 }
 
 // Wide (256 x 512) GEMM tiles when they cover the N columns with no more padding than
-// 256-wide tiles; their output column tile width.
-int gemm_wide(int64_t N) { return round_up(N, 2 * kBlockN) == round_up(N, kBlockN) ? 1 : 0; }
+// 256-wide tiles and still give every resident CTA pair a tile (`m_tiles`: 256-row tiles of
+// the launch); their output column tile width.
+int gemm_wide(int64_t N, int64_t m_tiles, int pairs) {
+  if (round_up(N, 2 * kBlockN) != round_up(N, kBlockN)) return 0;
+  return m_tiles * ((N + 2 * kBlockN - 1) / (2 * kBlockN)) >= pairs ? 1 : 0;
+}
 int gemm_tile_n(int wide) { return wide ? kWideN : kBlockN; }
 
 int sweep_units(const Layout& L, const SweepArgs& a) {
@@ -784,7 +788,8 @@ nb_status nb_kl_backward(const nb_kl_shape* shape, const void* h_s, const void* 
   GemmArgs g;
   std::memset(&g, 0, sizeof(g));
   g.nprob = 2;
-  g.wide = gemm_wide(L.d_s);
+  // 256-row tiles of one chunk's launch: dh_s (tokens) and dW_s (chunk columns)
+  g.wide = gemm_wide(L.d_s, L.N_pad / kPairM + (L.chunk_v + kPairM - 1) / kPairM, dev.pairs);
   g.n_valid = &w.ctrl->n_valid;
   g.status = &w.ctrl->status;
   g.wait_limit_ns = kWaitLimitNs;
@@ -891,7 +896,7 @@ nb_status nb_kl_gram(const void* X, int64_t rows, int64_t d, float* G, void* wor
   q.M = int(d);
   q.N = int(d);
   q.K = int(rows);
-  g.wide = gemm_wide(d);
+  g.wide = gemm_wide(d, (d + kPairM - 1) / kPairM, dev.pairs);
   const int tiles = int((d + kPairM - 1) / kPairM * ((d + gemm_tile_n(g.wide) - 1) / gemm_tile_n(g.wide)));
   next_cat(NB_KL_KERNEL_GEMM_PROJ);
   launch(gemm_kernel, dim3(pair_grid(dev, tiles)), dim3(kThreads), size_t(kSmemBytes), st, gm, g);
@@ -932,7 +937,7 @@ nb_status nb_kl_project(const void* X, int64_t rows, int64_t d, const void* B, i
   q.N = int(k);
   q.K = int(d);
   q.out_bf16 = 1;
-  g.wide = gemm_wide(k);
+  g.wide = gemm_wide(k, (rows + kPairM - 1) / kPairM, dev.pairs);
   const int tiles = int((rows + kPairM - 1) / kPairM * ((k + gemm_tile_n(g.wide) - 1) / gemm_tile_n(g.wide)));
   next_cat(NB_KL_KERNEL_GEMM_PROJ);
   launch(gemm_kernel, dim3(pair_grid(dev, tiles)), dim3(kThreads), size_t(kSmemBytes), st, gm, g);
@@ -1007,7 +1012,7 @@ nb_status nb_kl_debug_gemm(const void* A, int a_mn_major, const void* B, int b_m
   q.K = int(K);
   ok = make_out_map(&gm.out[0], C, N, M);
   if (!ok) return NB_ERR_CUDA;
-  g.wide = gemm_wide(N);
+  g.wide = gemm_wide(N, (M + kPairM - 1) / kPairM, dev.pairs);
   const int tiles = int((M + kPairM - 1) / kPairM * ((N + gemm_tile_n(g.wide) - 1) / gemm_tile_n(g.wide)));
   launch(gemm_kernel, dim3(pair_grid(dev, tiles)), dim3(kThreads), size_t(kSmemBytes), st, gm, g);
   return check_launch();

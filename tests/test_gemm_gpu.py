@@ -28,7 +28,9 @@ def run(A_bits, a_mn, B_bits, b_mn, M, N, K):
 @pytest.mark.parametrize("a_mn", [0, 1])
 @pytest.mark.parametrize("b_mn", [0, 1])
 @pytest.mark.parametrize("M,N,K", [(128, 128, 64), (256, 384, 320), (136, 264, 200), (1024, 512, 1000),
-                                   (304, 1288, 136), (520, 640, 512)])
+                                   (304, 1288, 136), (520, 640, 512),
+                                   # enough 256-row tiles for the 256 x 512 wide tiles (one per CTA pair)
+                                   (19200, 512, 200), (9480, 776, 136)])
 def test_gemm_layouts(a_mn, b_mn, M, N, K):
     rng = np.random.default_rng(M * 7 + N * 3 + K)
     A = f32_to_bf16_bits(rng.standard_normal((M, K)).astype(np.float32))

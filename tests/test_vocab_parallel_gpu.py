@@ -112,3 +112,10 @@ def test_full_size_sampled_rows(name, R):
     gu.check_forward(got, ref, x.labels, rows=sample)
     gu.check_side(got, ref, x.labels, x.W_s.shape[0], rows=sample)
     assert got["loss_mean"] == pytest.approx(got["loss_tok"].sum() / got["n_valid"], rel=1e-5)
+
+
+@pytest.mark.parametrize("R", [2, 3])
+def test_fp32_hidden_states(R):
+    """The 128-token workload (fp32 hidden states carried as bf16 hi + lo) with the vocabulary
+    split over R shards."""
+    check(make_inputs("tiny"), R)
