@@ -1,10 +1,15 @@
 // C-ABI host layer: argument checks, workspace carve-up, TMA descriptors, launches.
 //
 // One forward call: compaction of the valid rows -> vocabulary sweep (both block GEMMs,
-// online LSE / KL epilogue, split-V partial state) -> split-V merge -> [JSD: second
-// sweep with the final LSEs -> partial-sum reduction] -> masked mean.
+// online LSE / KL epilogue, split-V partial state; with side outputs also the student
+// entropy accumulator and the label logit) -> split-V merge -> [JSD: second sweep with the
+// final LSEs -> partial-sum reduction] -> masked mean.
 // One backward call: compaction -> per vocabulary chunk { gradient sweep writing the bf16
 // gradient chunk G; grouped GEMM dh_s (+)= G W_s[chunk], dW_s[chunk] (+)= G^T h_s }.
+// Vocabulary-parallel calls: the forward's sweep on one row shard of the unembeddings with
+// the merged shard state as output, the cross-shard merge, and the JSD's second pass per shard.
+// Spectral front end: Gram matrix and bf16 projections on the backward's GEMM kernel.
+// Hand-off: a row copy from peer or IPC-mapped memory.
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
