@@ -60,6 +60,19 @@ def _dist_all_reduce(group):
     return reduce
 
 
+def _check_device_f32(name, t, shape):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda or t.dtype != torch.float32 or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous float32 CUDA tensor")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}")
+
+
+def _check_labels(labels):
+    if not isinstance(labels, torch.Tensor) or not labels.is_cuda or labels.dtype != torch.int64 \
+            or labels.dim() != 1 or not labels.is_contiguous():
+        raise ValueError("labels must be a contiguous int64 CUDA tensor [N]")
+
+
 class LibraryKernels:
     """The library's calls on device tensors (the product path)."""
 
@@ -76,9 +89,11 @@ class LibraryKernels:
         return st, ws
 
     def combine(self, states, labels, beta, ignore_index, side):
+        _check_labels(labels)
         n_parts, N = states.shape[0], labels.shape[0]
-        if states.shape[1:] != (VP_FIELDS, N) or states.dtype != torch.float32 or not states.is_contiguous():
-            raise ValueError("states must be contiguous float32 [parts, VP_FIELDS, N]")
+        _check_device_f32("states", states, (n_parts, VP_FIELDS, N))
+        if states.device != labels.device:
+            raise ValueError("states and labels must be on the same device")
         f32 = dict(dtype=torch.float32, device=labels.device)
         out = {k: torch.empty(N, **f32) for k in ("loss_tok", "lse_s", "lse_t", "aux")}
         if side:
@@ -95,6 +110,9 @@ class LibraryKernels:
         return out
 
     def jsd_partial(self, h_s, W_s, h_t, W_t, labels, beta, tau, lse_s, lse_t, ignore_index, workspace=None):
+        _check_inputs(h_s, W_s, h_t, W_t, labels)
+        _check_device_f32("lse_s", lse_s, (labels.shape[0],))
+        _check_device_f32("lse_t", lse_t, (labels.shape[0],))
         shape = make_shape(h_s, W_s, h_t, W_t, labels, ignore_index)
         ws = _workspace(workspace_bytes(shape, beta), h_s.device, workspace)
         part = torch.empty((2, labels.shape[0]), dtype=torch.float32, device=h_s.device)
@@ -106,9 +124,11 @@ class LibraryKernels:
         return part
 
     def jsd_combine(self, parts, labels, ignore_index):
+        _check_labels(labels)
         n_parts, N = parts.shape[0], labels.shape[0]
-        if parts.shape[1:] != (2, N) or parts.dtype != torch.float32 or not parts.is_contiguous():
-            raise ValueError("parts must be contiguous float32 [parts, 2, N]")
+        _check_device_f32("parts", parts, (n_parts, 2, N))
+        if parts.device != labels.device:
+            raise ValueError("parts and labels must be on the same device")
         f32 = dict(dtype=torch.float32, device=labels.device)
         out = {"loss_tok": torch.empty(N, **f32), "aux": torch.empty(N, **f32),
                "loss_mean": torch.empty((), **f32),

@@ -177,3 +177,25 @@ def test_chunk_columns(L):
     # an explicit chunk is kept; an invalid shape gives 0
     assert lib.nb_kl_chunk_columns(L.shape_ptr(shape(L, chunk=4096))) == 4096
     assert lib.nb_kl_chunk_columns(L.shape_ptr(shape(L, ds=100))) == 0
+
+
+def test_python_layers_refuse_host_tensors(L):
+    """Every binding checks that its tensors are on the GPU before a pointer reaches the library."""
+    import torch
+    from full_vocab_kl_b200 import handoff, spectral
+    from full_vocab_kl_b200.vocab_parallel import LibraryKernels
+    k = LibraryKernels()
+    lab = torch.zeros(4, dtype=torch.int64)
+    with pytest.raises(ValueError):
+        k.combine(torch.zeros((2, L.VP_FIELDS, 4)), lab, 1.0, -100, False)
+    with pytest.raises(ValueError):
+        k.jsd_combine(torch.zeros((2, 2, 4)), lab, -100)
+    x = torch.zeros((4, 8), dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        k.jsd_partial(x, x, x, x, lab, 0.5, 1.0, torch.zeros(4), torch.zeros(4), -100)
+    with pytest.raises(ValueError):
+        spectral.gram(x)
+    with pytest.raises(ValueError):
+        spectral.project(x, torch.zeros((8, 8), dtype=torch.bfloat16))
+    with pytest.raises(ValueError):
+        handoff.receive_rows(x)
