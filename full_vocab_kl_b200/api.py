@@ -93,6 +93,17 @@ def kl_forward(h_s, W_s, h_t, W_t, labels, beta: float = 1.0, tau: float = 1.0, 
         if side:
             out["entropy_s"] = torch.empty(N, **f32)
             out["logp_label"] = torch.empty(N, **f32)
+    else:
+        # caller-supplied outputs: device tensors of the right dtype and shape
+        want = {"loss_tok": (torch.float32, (N,)), "lse_s": (torch.float32, (N,)), "lse_t": (torch.float32, (N,)),
+                "aux": (torch.float32, (N,)), "loss_mean": (torch.float32, ()), "n_valid": (torch.int64, ())}
+        if side:
+            want.update(entropy_s=(torch.float32, (N,)), logp_label=(torch.float32, (N,)))
+        for k, (dt, shp) in want.items():
+            t = out.get(k)
+            if not isinstance(t, torch.Tensor) or not t.is_cuda or t.device != dev or t.dtype != dt \
+                    or tuple(t.shape) != shp or not t.is_contiguous():
+                raise ValueError(f"out['{k}'] must be a contiguous {dt} tensor of shape {shp} on {dev}")
     common = (_abi.shape_ptr(shape), h_s.data_ptr(), W_s.data_ptr(), h_t.data_ptr(), W_t.data_ptr(),
               labels.data_ptr(), float(beta), float(tau), out["loss_tok"].data_ptr(), out["lse_s"].data_ptr(),
               out["lse_t"].data_ptr(), out["aux"].data_ptr(), out["loss_mean"].data_ptr(),

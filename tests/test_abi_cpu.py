@@ -199,3 +199,18 @@ def test_python_layers_refuse_host_tensors(L):
         spectral.project(x, torch.zeros((8, 8), dtype=torch.bfloat16))
     with pytest.raises(ValueError):
         handoff.receive_rows(x)
+
+
+def test_forward_out_dict_is_checked(L, monkeypatch):
+    """A caller-supplied output dictionary is validated before the call (here the inputs pass the
+    device check through a stand-in, and the outputs are host tensors)."""
+    import torch
+    from full_vocab_kl_b200 import api
+    monkeypatch.setattr(api, "_check_inputs", lambda *a: None)
+    monkeypatch.setattr(api, "_workspace", lambda n, dev, ws: None)
+    x = torch.zeros((4, 8), dtype=torch.bfloat16)
+    lab = torch.zeros(4, dtype=torch.int64)
+    out = {k: torch.zeros(4) for k in ("loss_tok", "lse_s", "lse_t", "aux")}
+    out.update(loss_mean=torch.zeros(()), n_valid=torch.zeros((), dtype=torch.int64))
+    with pytest.raises(ValueError):
+        api.kl_forward(x, x, x, x, lab, 1.0, 1.0, out=out)
