@@ -145,3 +145,20 @@ def test_vocab_tail_leaves_whole_column_halves_empty(V, beta):
     # lies entirely past the vocabulary, so some epilogue threads start on an all-masked chunk
     x = make_custom(300, 128, 192, V, beta, 0.7, n_masked=40, teacher="correlated")
     full_check(x)
+
+
+def test_empty_input():
+    """n_tokens = 0: loss 0, N_v 0, dW_s overwritten with zeros, no launch of a sweep."""
+    import torch
+    import full_vocab_kl_b200 as nb
+    z = lambda *s: torch.zeros(s, dtype=torch.bfloat16, device="cuda")  # noqa: E731
+    h_s, h_t, W_s, W_t = z(0, 128), z(0, 192), z(512, 128), z(512, 192)
+    lab = torch.zeros(0, dtype=torch.int64, device="cuda")
+    f = nb.kl_forward(h_s, W_s, h_t, W_t, lab, 0.5, 1.0, side=True)
+    dW = torch.full((512, 128), 3.0, device="cuda")
+    dh, dW = nb.kl_backward(h_s, W_s, h_t, W_t, lab, 0.5, 1.0, f["lse_s"], f["lse_t"], f["aux"], 1.0,
+                            dW_s=dW, workspace=f["workspace"])
+    torch.cuda.synchronize()
+    assert float(f["loss_mean"]) == 0.0 and int(f["n_valid"]) == 0
+    assert dh.shape == (0, 128) and float(dW.abs().max()) == 0.0
+    assert nb.device_status(f["workspace"]) == 0
