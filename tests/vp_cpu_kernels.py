@@ -46,6 +46,11 @@ class CpuKernels:
         return torch.from_numpy(st.astype(np.float32)), None
 
     def combine(self, states, labels, beta, ignore_index, side):
+        # masked rows hold zero states (l = 0); their values are computed and then discarded
+        with np.errstate(divide="ignore", invalid="ignore"):
+            return self._combine(states, labels, beta, ignore_index, side)
+
+    def _combine(self, states, labels, beta, ignore_index, side):
         S = _np(states).astype(np.float64)
         lab = _np(labels)
         N = lab.shape[0]
