@@ -1,0 +1,62 @@
+/* Host-side use of the C ABI from plain C99: the header compiles as C, the library links and
+ * loads, and the calls that need no GPU behave as the header states (sizes, status strings,
+ * synchronous argument errors). Prints "ok" and returns 0 on success. */
+#include <stdint.h>
+#include <stdio.h>
+#include <string.h>
+
+#include "nb_kl.h"
+
+#define CHECK(cond)                                                      \
+  do {                                                                   \
+    if (!(cond)) {                                                       \
+      fprintf(stderr, "check failed at line %d: %s\n", __LINE__, #cond); \
+      return 1;                                                          \
+    }                                                                    \
+  } while (0)
+
+int main(void) {
+  nb_kl_shape s;
+  memset(&s, 0, sizeof(s));
+  s.n_tokens = 8192;
+  s.vocab = 151936;
+  s.d_s = 1024;
+  s.d_t = 2560;
+  s.h_dtype = NB_BF16;
+  s.ignore_index = -100;
+
+  /* workspace: O(N * chunk), never O(N * V): well below one fp32 logit tensor, and doubling V
+   * adds at most the split-V state; the chunk follows the documented default */
+  const size_t ws = nb_kl_workspace_size(&s, 1.0f);
+  CHECK(ws > 0 && ws < (size_t)8192 * 151936 * 4 / 2);
+  nb_kl_shape big = s;
+  big.vocab = 2 * s.vocab;
+  CHECK(nb_kl_workspace_size(&big, 1.0f) - ws < (size_t)64 << 20);
+  CHECK(nb_kl_chunk_columns(&s) == 32768);
+  CHECK(nb_kl_workspace_size(&s, 0.5f) >= ws);
+
+  /* an invalid shape gives 0 */
+  nb_kl_shape bad = s;
+  bad.d_s = 100;
+  CHECK(nb_kl_workspace_size(&bad, 1.0f) == 0 && nb_kl_chunk_columns(&bad) == 0);
+
+  CHECK(strcmp(nb_kl_status_string(NB_OK), "ok") == 0);
+  CHECK(strcmp(nb_kl_status_string(NB_ERR_WORKSPACE), "workspace too small") == 0);
+
+  /* argument errors are returned synchronously, before any device work */
+  float f = 0.f;
+  int64_t n = 0;
+  void* p = (void*)(uintptr_t)0x10000; /* 16-byte aligned, never dereferenced */
+  CHECK(nb_kl_forward(&s, NULL, p, p, p, (const int64_t*)p, 1.0f, 1.0f, (float*)p, (float*)p, (float*)p,
+                      (float*)p, &f, &n, p, ws, NULL) == NB_ERR_INVALID_ARG);
+  CHECK(nb_kl_forward(&s, p, p, p, p, (const int64_t*)p, 1.5f, 1.0f, (float*)p, (float*)p, (float*)p,
+                      (float*)p, &f, &n, p, ws, NULL) == NB_ERR_INVALID_ARG);
+  CHECK(nb_kl_forward(&s, p, p, p, p, (const int64_t*)p, 1.0f, 1.0f, (float*)p, (float*)p, (float*)p,
+                      (float*)p, &f, &n, p, 100, NULL) == NB_ERR_WORKSPACE);
+  CHECK(nb_kl_vp_combine(8, 0, (const float*)p, (const int64_t*)p, -100, 1.0f, (float*)p, (float*)p, (float*)p,
+                         (float*)p, NULL, NULL, &f, &n, NULL) == NB_ERR_INVALID_ARG);
+  CHECK(nb_kl_project(p, 100, 64, p, 4, p, p, NULL) == NB_ERR_INVALID_ARG);
+  CHECK(nb_kl_handoff_rows(p, p, 10, 24, NULL, -100, NULL) == NB_ERR_INVALID_ARG);
+  printf("ok\n");
+  return 0;
+}

@@ -214,3 +214,22 @@ def test_forward_out_dict_is_checked(L, monkeypatch):
     out.update(loss_mean=torch.zeros(()), n_valid=torch.zeros((), dtype=torch.int64))
     with pytest.raises(ValueError):
         api.kl_forward(x, x, x, x, lab, 1.0, 1.0, out=out)
+
+
+def test_c_program_uses_the_abi(L, tmp_path):
+    """A plain C99 program compiled against include/nb_kl.h links the library and gets the
+    documented host-side behaviour (tests/c/abi_check.c)."""
+    import shutil
+    import subprocess
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("no C compiler")
+    from full_vocab_kl_b200 import build
+    libdir = os.path.dirname(build.LIB)
+    exe = str(tmp_path / "abi_check")
+    r = subprocess.run([gcc, "-std=c99", "-Wall", "-Werror", "-I", os.path.join(ROOT, "include"),
+                        os.path.join(ROOT, "tests", "c", "abi_check.c"), "-o", exe, "-L", libdir, "-lnbkl",
+                        "-Wl,-rpath," + libdir], capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+    r = subprocess.run([exe], capture_output=True, text=True, timeout=60)
+    assert r.returncode == 0 and r.stdout.strip() == "ok", r.stdout + r.stderr
