@@ -13,7 +13,8 @@ from hypothesis import strategies as st
 
 import oracle
 
-SETTINGS = settings(max_examples=40, deadline=None)
+# derandomized: the same examples on every run, so the CPU suite is reproducible
+SETTINGS = settings(max_examples=40, deadline=None, derandomize=True)
 
 
 def problem(seed, N, V, d_s, d_t, scale):
@@ -91,9 +92,11 @@ def test_gradient_is_linear_in_grad_out_and_rows_sum_to_zero(d, beta, tau, g):
     bg = oracle.backward(h_s, W_s, h_t, W_t, labels, beta, tau, grad_out=g)
     np.testing.assert_allclose(bg["dh_s"], g * b1["dh_s"], rtol=1e-12, atol=1e-14)
     np.testing.assert_allclose(bg["dW_s"], g * b1["dW_s"], rtol=1e-12, atol=1e-14)
+    # the row sums of G vanish only up to rounding of its terms (|G| |h| summed): an absolute
+    # floor far below any gradient a slip would leave behind
     col = np.abs(b1["dW_s"].sum(axis=0)).max()
     scale = np.abs(b1["dW_s"]).sum(axis=0).max() + 1e-300
-    assert col <= 1e-10 * scale + 1e-15
+    assert col <= 1e-10 * scale + 1e-13
 
 
 @SETTINGS
