@@ -181,29 +181,35 @@ def vp_backward(h_s, W_s_shard, h_t, W_t_shard, labels, beta: float, tau: float,
 
 class _VocabParallelKL(torch.autograd.Function):
     @staticmethod
-    def forward(ctx, h_s, W_s, h_t, W_t, labels, beta, tau, vocab_offset, group, ignore_index):
+    def forward(ctx, h_s, W_s, h_t, W_t, labels, beta, tau, vocab_offset, group, ignore_index, kernels, all_gather,
+                all_reduce):
         out = vp_forward(h_s, W_s, h_t, W_t, labels, beta, tau, vocab_offset=vocab_offset, group=group,
-                         ignore_index=ignore_index)
+                         ignore_index=ignore_index, kernels=kernels, all_gather=all_gather)
         ctx.save_for_backward(h_s, W_s, h_t, W_t, labels, out["lse_s"], out["lse_t"], out["aux"])
-        ctx.cfg = (beta, tau, group, ignore_index)
+        ctx.cfg = (beta, tau, group, ignore_index, kernels, all_reduce)
         ctx.workspace = out["workspace"]
         return out["loss_mean"]
 
     @staticmethod
     def backward(ctx, grad):
         h_s, W_s, h_t, W_t, labels, lse_s, lse_t, aux = ctx.saved_tensors
-        beta, tau, group, ignore_index = ctx.cfg
+        beta, tau, group, ignore_index, kernels, all_reduce = ctx.cfg
         dh, dW = vp_backward(h_s, W_s, h_t, W_t, labels, beta, tau, lse_s, lse_t, aux, grad, group=group,
-                             ignore_index=ignore_index, workspace=ctx.workspace)
-        return dh.to(h_s.dtype), dW.to(W_s.dtype), None, None, None, None, None, None, None, None
+                             ignore_index=ignore_index, kernels=kernels, workspace=ctx.workspace,
+                             all_reduce=all_reduce)
+        return (dh.to(h_s.dtype), dW.to(W_s.dtype)) + (None,) * 11
 
 
 def vocab_parallel_jsd(h_s, h_t, W_s_shard, W_t_shard, labels, vocab_offset: int, beta: float = 1.0,
-                       temperature: float = 1.0, group=None, ignore_index: int = IGNORE_INDEX):
+                       temperature: float = 1.0, group=None, ignore_index: int = IGNORE_INDEX, *,
+                       kernels=None, all_gather: Optional[Callable] = None,
+                       all_reduce: Optional[Callable] = None):
     """Scalar per-token-mean generalized JSD with row-sharded unembeddings; differentiable in
-    h_s (gradient summed over the ranks) and in this rank's W_s rows."""
+    h_s (gradient summed over the ranks) and in this rank's W_s rows. `kernels`, `all_gather`
+    and `all_reduce` default to the library and torch.distributed over `group`."""
     hs = h_s.reshape(-1, h_s.shape[-1]).contiguous()
     ht = h_t.reshape(-1, h_t.shape[-1]).contiguous()
     lab = labels.reshape(-1).contiguous()
     return _VocabParallelKL.apply(hs, W_s_shard.contiguous(), ht, W_t_shard.contiguous(), lab, float(beta),
-                                  float(temperature), int(vocab_offset), group, int(ignore_index))
+                                  float(temperature), int(vocab_offset), group, int(ignore_index), kernels,
+                                  all_gather, all_reduce)

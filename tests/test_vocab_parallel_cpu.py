@@ -144,3 +144,41 @@ def test_exchange_format_composes_for_any_split():
                                        err_msg=key)
 
     check()
+
+
+def _autograd_worker(rank, world, port, seed, beta, tau, out):
+    import torch
+    import torch.distributed as dist
+    from vp_cpu_kernels import CpuKernels
+    from full_vocab_kl_b200.vocab_parallel import vocab_parallel_jsd
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    h_s, W_s, h_t, W_t, labels = _problem(seed, beta=beta)
+    v0, v1 = shard_range(W_s.shape[0], rank, world, 16)
+    hs = torch.from_numpy(h_s).requires_grad_(True)
+    Ws = torch.from_numpy(W_s[v0:v1].copy()).requires_grad_(True)
+    loss = vocab_parallel_jsd(hs, torch.from_numpy(h_t), Ws, torch.from_numpy(W_t[v0:v1].copy()),
+                              torch.from_numpy(labels), v0, beta, tau, kernels=CpuKernels())
+    (0.8 * loss).backward()
+    out[rank] = {"loss": float(loss), "dh": hs.grad.numpy(), "dW": Ws.grad.numpy(), "range": (v0, v1)}
+    dist.barrier()
+    dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("beta", [1.0, 0.5])
+def test_autograd_through_the_sharded_loss(beta):
+    """loss.backward() on every rank: dh_s summed over the ranks, dW_s for the rank's own rows."""
+    seed, world, tau = 3, 2, 1.3
+    port = _free_port()
+    mgr = mp.get_context("spawn").Manager()
+    out = mgr.dict()
+    mp.start_processes(_autograd_worker, args=(world, port, seed, beta, tau, out), nprocs=world, join=True,
+                       start_method="spawn")
+    h_s, W_s, h_t, W_t, labels = _problem(seed, beta=beta)
+    ref = oracle.forward(h_s, W_s, h_t, W_t, labels, beta, tau)
+    refb = oracle.backward(h_s, W_s, h_t, W_t, labels, beta, tau, grad_out=0.8)
+    for r in range(world):
+        assert out[r]["loss"] == pytest.approx(ref["loss_mean"], rel=2e-5)
+        np.testing.assert_allclose(out[r]["dh"], refb["dh_s"], rtol=1e-4, atol=1e-7)
+        v0, v1 = out[r]["range"]
+        np.testing.assert_allclose(out[r]["dW"], refb["dW_s"][v0:v1], rtol=1e-4, atol=1e-7)
