@@ -79,13 +79,21 @@ def algorithmic_flops(w, n_valid, V=None, proj=0.0):
 PROFILED_SOURCES = ("common.cuh", "gemm.cuh", "ptx.cuh", "sweep.cuh")
 
 
+def _code_only(text: str) -> str:
+    """C++ source without comments and with whitespace collapsed: what the compiler sees."""
+    text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", " ", text)
+    return " ".join(text.split())
+
+
 def kernel_source_sha():
-    """Hash of the sweep and GEMM device code: a profile summary is only used while it matches."""
+    """Hash of the sweep and GEMM device code (comments and layout ignored): a profile summary
+    is only used while it matches."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "full_vocab_kl_b200", "csrc")
     for name in PROFILED_SOURCES:
-        with open(os.path.join(csrc, name), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(csrc, name), encoding="utf-8") as f:
+            h.update(_code_only(f.read()).encode())
     return h.hexdigest()[:16]
 
 

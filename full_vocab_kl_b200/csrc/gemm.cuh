@@ -11,8 +11,10 @@
 //
 // A pair of CTAs computes a 256 x 256 output tile (cta_group::2): each CTA stages its 128 rows
 // of A and 128 of the 256 columns of B, and holds its 128 output rows (one 256-column fp32
-// accumulator, double-buffered in TMEM). Same warp roles and barriers as the sweep; warps
-// 4-11 write one output row half (128 columns) per thread.
+// accumulator, double-buffered in TMEM). Wide launches use 256 x 512 tiles instead: both TMEM
+// buffers hold one tile, each stage carries A and two B halves, and the epilogue reads the tile
+// as two 256-column halves. Same warp roles and barriers as the sweep; warps 4-11 write one
+// output row half (128 columns) per thread.
 #pragma once
 
 #include "common.cuh"

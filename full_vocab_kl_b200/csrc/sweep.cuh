@@ -35,7 +35,7 @@
 namespace nbkl {
 
 struct SweepSmem {
-  uint8_t* a;           // kStages x 16 KB
+  uint8_t* a;           // kStages x 16 KB (wide GEMM tiles: a and b together as 4 x 48 KB)
   uint8_t* b;           // kStages x 16 KB
   uint8_t* out;         // kEpiWarps x 4 KB TMA-store staging
   uint64_t* full;       // kStages (leader: TMA bytes of both CTAs)
