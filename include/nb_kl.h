@@ -25,9 +25,11 @@
  * [n_tokens] int64; every per-token output [n_tokens] fp32; dh_s [n_tokens, d_s] fp32;
  * dW_s [vocab, d_s] fp32. Row n of h_s, h_t and labels is one position (no shift).
  *
- * Requirements (NB_ERR_INVALID_ARG otherwise): d_s and d_t multiples of 8; h_*, W_*
- * and the workspace 16-byte aligned; 0 <= beta <= 1; tau > 0 and finite;
- * workspace_bytes >= nb_kl_workspace_size(shape, beta). n_tokens may be 0.
+ * Requirements (NB_ERR_INVALID_ARG otherwise): d_s and d_t multiples of 8 in [8, 65536];
+ * 1 <= vocab <= 2^30; 0 <= n_tokens <= 2^30 (n_tokens may be 0); reserved == 0; chunk_v a
+ * multiple of 256 or 0; h_*, W_* and the workspace 16-byte aligned; 0 <= beta <= 1; tau > 0
+ * and finite. A workspace smaller than nb_kl_workspace_size(shape, beta) gives
+ * NB_ERR_WORKSPACE.
  *
  * Errors: invalid arguments are reported synchronously by the return value and launch
  * nothing. Device-side failures (a bounded wait that ran out) are written to a status
@@ -69,7 +71,7 @@ typedef struct nb_kl_shape {
   int32_t h_dtype;      /* nb_dtype of h_s and h_t; W_s and W_t are always bf16 */
   int32_t reserved;     /* must be 0 */
   int64_t ignore_index; /* label of masked positions, normally -100 */
-  int64_t chunk_v;      /* backward vocabulary chunk (multiple of 128); 0 = library default */
+  int64_t chunk_v;      /* backward vocabulary chunk (multiple of 256); 0 = library default */
 } nb_kl_shape;
 
 /* Bytes of scratch the calls need for this shape: O(n_tokens * (d_s + d_t + chunk_v))
