@@ -137,13 +137,13 @@ NB_KL_API nb_status nb_kl_forward_side(const nb_kl_shape* shape, const void* h_s
 #define NB_KL_VP_FIELDS 7
 
 /* First part on one shard. shape->vocab is the shard's row count; the workspace is sized by
- * nb_kl_workspace_size(shape, beta). Labels keep their global values. */
+ * nb_kl_workspace_size(shape, beta). Labels keep their global values. 0 <= vocab_offset <= 2^30. */
 NB_KL_API nb_status nb_kl_vp_state(const nb_kl_shape* shape, int64_t vocab_offset, const void* h_s,
                          const void* W_s, const void* h_t, const void* W_t, const int64_t* labels, float beta,
                          float tau, float* state, void* workspace, size_t workspace_bytes, void* stream);
 
-/* Merge of n_parts gathered shard states (device, [n_parts][NB_KL_VP_FIELDS][n_tokens]) in
- * part order, in fp64. Outputs as nb_kl_forward_side (entropy_s / logp_label may be NULL);
+/* Merge of n_parts (1 to 4096) gathered shard states (device, [n_parts][NB_KL_VP_FIELDS][n_tokens])
+ * in part order, in fp64. Outputs as nb_kl_forward_side (entropy_s / logp_label may be NULL);
  * for 0 < beta < 1, loss_tok and aux are written as 0 and loss_mean / n_valid are those of
  * the zero losses: nb_kl_vp_jsd_combine replaces them. No workspace. */
 NB_KL_API nb_status nb_kl_vp_combine(int64_t n_tokens, int n_parts, const float* states, const int64_t* labels,
@@ -198,7 +198,7 @@ NB_KL_API nb_status nb_kl_project(const void* X, int64_t rows, int64_t d, const 
  * with plain 16-byte loads (no TMA, no multicast) and writes dst (local, [n_rows, row_bytes]);
  * with labels (device int64 [n_rows]) only rows whose label is not ignore_index cross the link
  * and the other dst rows keep their contents. Both pointers 16-byte aligned, row_bytes a
- * multiple of 16. The loss can also take src directly as h_t: its row gather then reads the
+ * multiple of 16 (at most 2^24). The loss can also take src directly as h_t: its row gather then reads the
  * valid rows over the link in each call (forward and backward), where one hand-off into local
  * memory reads them once. */
 NB_KL_API nb_status nb_kl_handoff_rows(const void* src, void* dst, int64_t n_rows, int64_t row_bytes,
