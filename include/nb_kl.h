@@ -198,9 +198,9 @@ NB_KL_API nb_status nb_kl_project(const void* X, int64_t rows, int64_t d, const 
  * with plain 16-byte loads (no TMA, no multicast) and writes dst (local, [n_rows, row_bytes]);
  * with labels (device int64 [n_rows]) only rows whose label is not ignore_index cross the link
  * and the other dst rows keep their contents. Both pointers 16-byte aligned, row_bytes a
- * multiple of 16 (at most 2^24). The loss can also take src directly as h_t: its row gather then reads the
- * valid rows over the link in each call (forward and backward), where one hand-off into local
- * memory reads them once. */
+ * multiple of 16 (at most 2^24). The loss can also take src directly as h_t: its row gather
+ * then reads the valid rows over the link in each call (forward and backward), where one
+ * hand-off into local memory reads them once. */
 NB_KL_API nb_status nb_kl_handoff_rows(const void* src, void* dst, int64_t n_rows, int64_t row_bytes,
                              const int64_t* labels, int64_t ignore_index, void* stream);
 
