@@ -75,6 +75,13 @@ def algorithmic_flops(w, n_valid, V=None, proj=0.0):
     }
 
 
+def model_flops(w, n_valid, V=None) -> float:
+    """The stricter count with no recompute: one forward sweep over both models plus the dh_s and
+    dW_s products (the JSD's second sweep and the backward's recompute sweep are left out)."""
+    V = w.V if V is None else V
+    return 2.0 * n_valid * V * (w.d_s + w.d_t) + 4.0 * n_valid * V * w.d_s
+
+
 # headers that define the profiled tensor-core kernels (the vocabulary sweep and the GEMM)
 PROFILED_SOURCES = ("common.cuh", "gemm.cuh", "ptx.cuh", "sweep.cuh")
 
@@ -514,6 +521,7 @@ def run_library(args):
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded; shapes of the workload)",
             "config": config,
             "tflops": tflops, "pct_bf16_peak_datasheet": 100.0 * tflops / DATASHEET_BF16_TFLOPS,
+            "model_tflops": model_flops(w, n_valid, V_rank) * world / (ms_step * 1e-3) / 1e12,
             "pct_bf16_peak_measured": 100.0 * tflops / peaks.get("bf16_tflops", FALLBACK["bf16_tflops"]),
             "roofline": {"bound": "tensor", "kernel": dom, "achieved": achieved, "peak": peak,
                          "peak_source": f"{peak_src} bf16_tflops_sustained", "unit": "TFLOP/s",

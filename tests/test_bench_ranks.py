@@ -70,3 +70,19 @@ def test_reference_arm_line_on_rank0(monkeypatch, capsys):
     assert d["e2e"] == {"value": d["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0,
                         "d2h_bytes_per_step": 0}
     assert d["config"]["workload"] == "tiny"
+
+
+def test_flop_counts():
+    """Algorithmic FLOPs count the recompute; model FLOPs do not (OPD workload numbers)."""
+    import bench
+    from synthetic import WORKLOADS
+    w = WORKLOADS["opd_0p6b_4b"]
+    f = bench.algorithmic_flops(w, 4916)
+    sweep = 2.0 * 4916 * 151936 * (1024 + 2560)
+    assert f["sweep_fwd"] == f["sweep_grad"] == sweep and f["sweep_jsd"] == 0.0
+    assert f["gemm_bwd"] == 4.0 * 4916 * 151936 * 1024
+    assert sum(f.values()) == pytest.approx(13.77e12, rel=1e-3)
+    assert bench.model_flops(w, 4916) == pytest.approx(sum(f.values()) - sweep, rel=1e-12)
+    jsd = WORKLOADS["long_jsd"]
+    fj = bench.algorithmic_flops(jsd, 6144)
+    assert fj["sweep_jsd"] == fj["sweep_fwd"] > 0
