@@ -145,6 +145,20 @@ def _check(beta: float, tau: float):
         raise ValueError("tau must be positive")
 
 
+def _selected_rows(labels: np.ndarray, ignore_index: int, rows: Optional[Sequence[int]]):
+    """Valid mask, the valid positions to evaluate (all, or those of ``rows``), and N_v.
+
+    N_v counts every position whose label is not ``ignore_index`` ("03 White-box OPD",
+    section 2.3): it is the denominator of the per-token mean whether or not ``rows``
+    restricts the positions evaluated.
+    """
+    valid = labels != ignore_index
+    n_valid = int(valid.sum())
+    todo = np.flatnonzero(valid) if rows is None else np.asarray(
+        [r for r in rows if valid[r]], dtype=np.int64)
+    return valid, todo, n_valid
+
+
 def _row_blocks(rows: np.ndarray, block: int):
     for i in range(0, len(rows), block):
         yield rows[i:i + block]
@@ -164,10 +178,7 @@ def forward(h_s, W_s, h_t, W_t, labels, beta: float, tau: float, *,
     _check(beta, tau)
     labels = np.asarray(labels)
     N = labels.shape[0]
-    valid = labels != ignore_index
-    n_valid = int(valid.sum())
-    todo = np.flatnonzero(valid) if rows is None else np.asarray(
-        [r for r in rows if valid[r]], dtype=np.int64)
+    valid, todo, n_valid = _selected_rows(labels, ignore_index, rows)
     keys = ("loss_tok", "lse_s", "lse_t", "aux") + (("entropy_s", "logp_label") if side else ())
     out = {k: np.zeros(N) for k in keys}
     for r in _row_blocks(todo, row_block):
@@ -178,7 +189,7 @@ def forward(h_s, W_s, h_t, W_t, labels, beta: float, tau: float, *,
         out["lse_s"][r], out["lse_t"][r] = lse_s, lse_t
         if side:
             out["entropy_s"][r], out["logp_label"][r] = student_side_rows(logS, labels[r])
-    complete = len(todo) == n_valid
+    complete = np.unique(todo).size == n_valid   # every valid position was evaluated
     out["n_valid"] = n_valid
     if not complete:
         out["loss_mean"] = None
@@ -203,10 +214,7 @@ def backward(h_s, W_s, h_t, W_t, labels, beta: float, tau: float, *, grad_out: f
     _check(beta, tau)
     labels = np.asarray(labels)
     N, d_s = labels.shape[0], h_s.shape[1]
-    valid = labels != ignore_index
-    n_valid = int(valid.sum())
-    todo = np.flatnonzero(valid) if rows is None else np.asarray(
-        [r for r in rows if valid[r]], dtype=np.int64)
+    _, todo, n_valid = _selected_rows(labels, ignore_index, rows)
     want_dW = want_dW and rows is None
     dh = np.zeros((N, d_s))
     dW = None

@@ -186,3 +186,37 @@ def test_unscaled_teacher_unembedding_caught(monkeypatch):
         return hp, Wp / np.linalg.norm(Wp, axis=0, keepdims=True), Vk
     monkeypatch.setattr(spo, "compress_teacher", bad)
     assert _fails(spec_pins.test_closed_form_diagonal)
+
+
+# ------------------------------------------------------------------ partial paths
+import test_oracle_subset_pins as subset_pins  # noqa: E402
+
+
+def test_dropped_dW_init_caught(monkeypatch):
+    # an accumulating backward that starts dW_s from zero instead of the caller's start value
+    orig = ko.backward
+
+    def bad(*a, dW_init=None, **k):
+        return orig(*a, **k)
+
+    monkeypatch.setattr(subset_pins.oracle, "backward", bad)
+    assert _fails(subset_pins.test_dW_init_is_added_to_the_gradient, 1.0)
+
+
+def test_mean_over_sampled_rows_caught(monkeypatch):
+    # normalising by the number of positions evaluated instead of N_v
+    orig = ko._selected_rows
+
+    def bad(labels, ignore_index, rows):
+        valid, todo, _ = orig(labels, ignore_index, rows)
+        return valid, todo, int(todo.size)
+
+    monkeypatch.setattr(ko, "_selected_rows", bad)
+    assert _fails(subset_pins.test_rows_subset_backward_uses_all_valid_rows, 0.35)
+
+
+def test_rows_subset_ignored_caught(monkeypatch):
+    # a forward that evaluates every valid position whatever `rows` says
+    orig = ko._selected_rows
+    monkeypatch.setattr(ko, "_selected_rows", lambda labels, ii, rows: orig(labels, ii, None))
+    assert _fails(subset_pins.test_rows_subset_forward_matches_brute_force, 1.0)
