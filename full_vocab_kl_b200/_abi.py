@@ -45,6 +45,8 @@ SIGNATURES = {
                                      c_void_p, c_void_p]),
     "nb_kl_gram": (c_int, [c_void_p, c_int64, c_int64, c_void_p, c_void_p, c_void_p]),
     "nb_kl_project": (c_int, [c_void_p, c_int64, c_int64, c_void_p, c_int64, c_void_p, c_void_p, c_void_p]),
+    "nb_kl_spectral_select": (c_int, [c_void_p, c_void_p, c_int64, c_int64, c_void_p, c_void_p, c_void_p,
+                                      c_void_p]),
     "nb_kl_handoff_rows": (c_int, [c_void_p, c_void_p, c_int64, c_int64, c_void_p, c_int64, c_void_p]),
     "nb_kl_enable_peer_access": (c_int, [c_int]),
     "nb_kl_backward": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_float, c_float,
@@ -53,6 +55,7 @@ SIGNATURES = {
     "nb_kl_forward_noalloc": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_float,
                                       c_float, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
                                       c_void_p]),
+    "nb_kl_noalloc_device_status": (c_int, [c_void_p]),
     "nb_kl_status_string": (c_char_p, [c_int]),
     "nb_kl_device_status": (c_int, [c_void_p, c_void_p]),
     "nb_kl_debug_gemm": (c_int, [c_void_p, c_int, c_void_p, c_int, c_int64, c_int64, c_int64, c_void_p, c_void_p,

@@ -20,10 +20,13 @@ constexpr int kPairM = 2 * kBlockM;                    // rows per pair (MMA M)
 constexpr int kBlockN = 256;                           // MMA N
 constexpr int kHalfB = kBlockN / 2;                    // B rows staged per CTA
 constexpr int kBlockK = 64;
+// Pipeline stages: 6 for the kernels that also stage output tiles for TMA stores (gradient
+// sweep, GEMM), 7 for the state and JSD sweeps, whose 7th stage takes the output staging area.
 constexpr int kStages = 6;
+constexpr int kMaxStages = 7;
 constexpr int kATileBytes = kBlockM * kBlockK * 2;     // 16 KB
 constexpr int kBTileBytes = kHalfB * kBlockK * 2;      // 16 KB
-constexpr int kStageBytes = kATileBytes + kBTileBytes; // 32 KB per CTA
+constexpr int kStageBytes = kATileBytes + kBTileBytes; // 32 KB per CTA: A tile, then B tile
 constexpr int kPairStageBytes = 2 * kStageBytes;       // bytes the leader's full barrier expects
 constexpr int kEpiWarps = 8;                           // two warps per TMEM lane quarter
 constexpr int kEpiWarp0 = 4;                           // epilogue = warpgroups 1 and 2
@@ -39,7 +42,9 @@ constexpr int kHalfN = kBlockN / 2;                    // columns per epilogue t
 // Per epilogue warp, one 4 KB staging buffer for TMA stores (32 rows x 128 bytes, 128-byte
 // swizzle: fp32 32 x 32 chunks of the GEMM output, bf16 32 x 32 chunks of the gradient).
 constexpr int kStageOutBytes = 4096;
-constexpr int kSmemBytes = kStages * kStageBytes + kEpiWarps * kStageOutBytes + 1024 /*align*/ + 256 /*barriers*/;
+static_assert(kStages * kStageBytes + kEpiWarps * kStageOutBytes <= kMaxStages * kStageBytes,
+              "output staging fits in the 7th stage");
+constexpr int kSmemBytes = kMaxStages * kStageBytes + 1024 /*align*/ + 256 /*barriers*/;
 
 constexpr int kRing = 4;                               // work ids in flight inside a pair
 constexpr int kRingConsumers = 2 * (1 + 8);            // per CTA: MMA or TMA thread + 8 epilogue warps
@@ -77,7 +82,8 @@ struct SweepArgs {
   int v_begin, v_end;     // vocabulary columns covered by this launch
   int nkb_s, nkb_t;       // K blocks of the A operands (student, teacher)
   int bmod_s, bmod_t;     // B block of A block kb is kb % bmod (fp32 hi/lo split reuses W)
-  int tiles_per_unit;     // vocabulary tiles per work unit (one split of the LSE state)
+  int tiles_per_unit;     // vocabulary tiles per work unit of the first n_big units (one split of the
+  int n_big;              // LSE state each); every later unit is a single tile (a short tail of work)
   float scale;            // log2(e) / tau: base-2 tempered logits x = z * scale
   float beta;
   float* out;             // state [6][split][ld] or JSD partial sums [2][split][ld]; split =
@@ -111,7 +117,7 @@ struct GemmProb {
   int a_koff, b_koff;      // K coordinate offsets of the operands
   int m_dyn, M;            // m_dyn: M = n_valid (else M)
   int N;
-  int k_dyn, K;            // k_dyn: K = round_up(n_valid, 128) (else K)
+  int k_dyn, K;            // k_dyn: K = round_up(n_valid, 64) (else K)
   int out_row0;            // output-map row of tile row 0
   int accumulate;          // 1: out += acc (TMA reduce-add), 0: out = acc (TMA store)
   int out_bf16;            // 1: out is bf16 (32 x 32 boxes, 64-byte swizzle), stored rounded to nearest even

@@ -28,7 +28,9 @@ struct TileInfo {
 
 __device__ __forceinline__ int prob_M(const GemmProb& q, int nv) { return q.m_dyn ? nv : q.M; }
 __device__ __forceinline__ int prob_K(const GemmProb& q, int nv) {
-  return q.k_dyn ? ((nv + kPairM - 1) / kPairM) * kPairM : q.K;
+  // rows n_valid .. (last 256-row tile) of the compacted operands are zeros: K stops at the K
+  // block that holds the last valid row
+  return q.k_dyn ? ((nv + kBlockK - 1) / kBlockK) * kBlockK : q.K;
 }
 __device__ __forceinline__ int prob_tiles(const GemmProb& q, int nv, int tile_n) {
   return ((prob_M(q, nv) + kPairM - 1) / kPairM) * ((q.N + tile_n - 1) / tile_n);
@@ -60,14 +62,13 @@ __device__ __forceinline__ int total_tiles(const GemmArgs& p, int nv) {
   return t;
 }
 
-// Shared-memory addresses of stage `st`'s operands: narrow tiles keep A and B in two arrays
-// of kStages x 16 KB; wide tiles use the same 192 KB as kWideStages x (A, B half 0, B half 1).
+// Shared-memory addresses of stage `st`'s operands: narrow tiles use kStages x (A, B) of 32 KB;
+// wide tiles use the same 192 KB as kWideStages x (A, B half 0, B half 1).
 __device__ __forceinline__ uint32_t stage_a(const SweepSmem& s, int wide, int st) {
-  return wide ? smem_addr(s.a + st * kWideStageBytes) : smem_addr(s.a + st * kATileBytes);
+  return wide ? smem_addr(s.a + st * kWideStageBytes) : stage_a_addr(s, st);
 }
 __device__ __forceinline__ uint32_t stage_b(const SweepSmem& s, int wide, int st, int half) {
-  return wide ? smem_addr(s.a + st * kWideStageBytes + kATileBytes + half * kBTileBytes)
-              : smem_addr(s.b + st * kBTileBytes);
+  return wide ? smem_addr(s.a + st * kWideStageBytes + kATileBytes + half * kBTileBytes) : stage_b_addr(s, st);
 }
 
 // K-major operand: one (rows x 64) box. MN-major operand: (rows / 64) boxes of 64 x 64
@@ -122,8 +123,8 @@ __device__ __forceinline__ void gemm_producer(const GemmMaps& maps, const GemmAr
       if (p.wide)   // the second 256-column half of the tile: this CTA's 128 of its B rows
         load_operand(stage_b(s, 1, stage, 1), &maps.b[ti.prob], bar, q.b_mn, bn0 + kBlockN, q.b_koff + kc,
                      kHalfB);
-      pend_stage[n_issued % kStages] = stage;
-      pend_par[n_issued % kStages] = phase;
+      pend_stage[n_issued % n_stages] = stage;
+      pend_par[n_issued % n_stages] = phase;
       ++n_issued;
       if (++stage == n_stages) { stage = 0; phase ^= 1u; }
     }

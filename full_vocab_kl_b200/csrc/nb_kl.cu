@@ -33,6 +33,7 @@ namespace {
 
 constexpr unsigned long long kWaitLimitNs = 1000000000ull;  // 1 s per pipeline wait
 constexpr int kTilesPerUnitFwd = 8;                          // 2048 vocabulary columns per unit
+constexpr int kTailItems = 160;   // single-tile work items at the end of a forward sweep (~2 waves of pairs)
 constexpr size_t kCtrlBytes = 256;
 
 thread_local int g_launches = 0;
@@ -69,6 +70,7 @@ struct Layout {
   int kb_s, kb_t;        // 64-wide K blocks of W
   int64_t lda_s, lda_t;  // row length of the compacted h buffers
   int n_vt, n_split;
+  int n_big;             // forward sweeps: vocabulary units of kTilesPerUnitFwd tiles (the rest are single tiles)
   int64_t chunk_v;
   int n_chunks;          // backward vocabulary chunks
   size_t off_idx, off_hs, off_ht, off_rl2s, off_rl2t, off_raux, off_rlab, off_labx, off_sched, off_dhc, off_state,
@@ -96,14 +98,22 @@ bool make_layout(const nb_kl_shape* sh, float beta, Layout& L) {
   L.lda_s = int64_t(L.kb_s) * kBlockK * (L.split ? 2 : 1);
   L.lda_t = int64_t(L.kb_t) * kBlockK * (L.split ? 2 : 1);
   L.n_vt = int((L.V + kBlockN - 1) / kBlockN);
-  L.n_split = 2 * ((L.n_vt + kTilesPerUnitFwd - 1) / kTilesPerUnitFwd);  // two column halves per unit
-  // default chunk: about 8192 gradient tiles of 128 x 256 per sweep launch (the two gradient
-  // buffers then take ~1 GB whatever the token count; longer chunks mean fewer launches and
-  // fewer re-adds of the compacted dh accumulator), but at least 4 d_s columns; between 2048
-  // and 32768 columns
-  const int64_t by_tiles = (int64_t(1) << 21) / (L.N_pad / kBlockM);
+  // forward units: runs of kTilesPerUnitFwd tiles, then enough single tiles that the last
+  // ~kTailItems work items (over all 256-row token tiles) are short
+  {
+    const int64_t n_tt = L.N_pad / kPairM;
+    const int n_single = int(std::min<int64_t>(L.n_vt, (kTailItems + n_tt - 1) / n_tt));
+    L.n_big = (L.n_vt - n_single) / kTilesPerUnitFwd;
+    const int n_vu = L.n_big + (L.n_vt - L.n_big * kTilesPerUnitFwd);
+    L.n_split = 2 * n_vu;  // two column halves per unit
+  }
+  // default chunk: about 16384 gradient tiles of 128 x 256 per sweep launch (the gradient
+  // buffer then takes ~1 GB whatever the token count; longer chunks mean fewer launches, shorter
+  // launch tails and fewer re-adds of the compacted dh accumulator), but at least 4 d_s columns;
+  // between 2048 and 65536 columns
+  const int64_t by_tiles = (int64_t(1) << 22) / (L.N_pad / kBlockM);
   const int64_t auto_chunk =
-      round_up(std::max<int64_t>(2048, std::min<int64_t>(32768, std::max<int64_t>(by_tiles, 4 * L.d_s))), kBlockN);
+      round_up(std::max<int64_t>(2048, std::min<int64_t>(65536, std::max<int64_t>(by_tiles, 4 * L.d_s))), kBlockN);
   L.chunk_v = sh->chunk_v ? sh->chunk_v : std::min<int64_t>(auto_chunk, round_up(L.V, kBlockN));
   const bool jsd = beta > 0.f && beta < 1.f;
   size_t off = kCtrlBytes;
@@ -118,14 +128,14 @@ bool make_layout(const nb_kl_shape* sh, float beta, Layout& L) {
   L.n_chunks = int((L.V + L.chunk_v - 1) / L.chunk_v);
   L.off_sched = off; off = align256(off + size_t(2 * L.n_chunks + 2) * 4);   // one work counter per launch
   L.off_dhc = off;   off = align256(off + size_t(L.N_pad) * L.d_s * 4);        // compacted dh_s (backward)
-  // the forward's split state and the backward's two gradient-chunk buffers share one region
+  // the forward's split state and the backward's gradient-chunk buffer share one region
   const size_t state_bytes = align256(size_t(6) * L.n_split * L.N_pad * 4);
   const size_t part_bytes = jsd ? align256(size_t(2) * L.n_split * L.N_pad * 4) : 0;
   L.g_bytes = align256(size_t(L.N_pad) * L.chunk_v * 2);
   L.off_state = off;
   L.off_part = off + state_bytes;
   L.off_G = off;
-  off += std::max(state_bytes + part_bytes, 2 * L.g_bytes);
+  off += std::max(state_bytes + part_bytes, L.g_bytes);
   L.total = off;
   L.fs_state = (long long)L.n_split * L.N_pad;
   return true;
@@ -154,27 +164,6 @@ struct DevInfo {
   bool attrs = false;
 };
 
-// Second stream of the backward (the GEMMs of chunk c overlap the gradient sweep of chunk
-// c + 1) and its events: one set per host thread and device, created on first use.
-struct AuxStream {
-  cudaStream_t aux = nullptr;
-  cudaEvent_t fork = nullptr, join = nullptr, swept[2] = {nullptr, nullptr}, used[2] = {nullptr, nullptr};
-};
-thread_local AuxStream g_aux[64];
-
-nb_status aux_stream(AuxStream** out) {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return NB_ERR_CUDA;
-  AuxStream& a = g_aux[dev];
-  if (!a.aux) {
-    if (cudaStreamCreateWithFlags(&a.aux, cudaStreamNonBlocking) != cudaSuccess) return NB_ERR_CUDA;
-    cudaEvent_t* evs[] = {&a.fork, &a.join, &a.swept[0], &a.swept[1], &a.used[0], &a.used[1]};
-    for (cudaEvent_t* e : evs)
-      if (cudaEventCreateWithFlags(e, cudaEventDisableTiming) != cudaSuccess) return NB_ERR_CUDA;
-  }
-  *out = &a;
-  return NB_OK;
-}
 DevInfo g_dev[64];
 std::mutex g_dev_mu;
 
@@ -350,6 +339,7 @@ SweepArgs base_sweep_args(const Layout& L, const Ws& w, float beta, float tau) {
   a.bmod_s = L.kb_s;
   a.bmod_t = L.kb_t;
   a.tiles_per_unit = kTilesPerUnitFwd;
+  a.n_big = L.n_big;
   a.scale = float(1.4426950408889634 / double(tau));
   a.beta = beta;
   a.ld = int(L.N_pad);
@@ -381,7 +371,7 @@ int gemm_tile_n(int wide) { return wide ? kWideN : kBlockN; }
 int sweep_units(const Layout& L, const SweepArgs& a) {
   const int n_tt = int(L.N_pad / kPairM);
   const int n_vt = (a.v_end - a.v_begin + kBlockN - 1) / kBlockN;
-  const int n_vu = (n_vt + a.tiles_per_unit - 1) / a.tiles_per_unit;
+  const int n_vu = a.n_big + (n_vt - a.n_big * a.tiles_per_unit);
   return n_tt * n_vu;
 }
 
@@ -766,30 +756,29 @@ nb_status nb_kl_backward(const nb_kl_shape* shape, const void* h_s, const void* 
          dh_s, int(L.d_s));
 
   if (cudaMemsetAsync(w.sched, 0, size_t(2 * L.n_chunks + 2) * 4, st) != cudaSuccess) return NB_ERR_CUDA;
-  // two gradient-chunk buffers: the sweep of chunk c + 1 may run while the GEMMs of chunk c read
-  __nv_bfloat16* gbuf[2] = {w.G, reinterpret_cast<__nv_bfloat16*>(reinterpret_cast<uint8_t*>(w.G) + L.g_bytes)};
-  SweepMaps maps[2];
-  GemmMaps gm[2];
-  bool ok = true;
-  for (int b = 0; b < 2; ++b) {
-    ok &= sweep_maps(L, w, W_s, W_t, maps[b]);
-    // gradient chunk written by the sweep epilogue: bf16 32 x 32 boxes, 64-byte rows
-    ok &= make_map(&maps[b].g_out, gbuf[b], L.chunk_v, L.N_pad, L.chunk_v * 2, 32, 32,
-                   CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, CU_TENSOR_MAP_SWIZZLE_64B);
-    ok &= make_out_map(&gm[b].out[0], w.dhc, L.d_s, L.N_pad);
-    ok &= make_out_map(&gm[b].out[1], dW_s, L.d_s, L.V);
-    // dh_s: A = G (K-major, box 64 x 128), B = W_s chunk as K x N (MN-major, 64 x 64 boxes)
-    ok &= make_map(&gm[b].a[0], gbuf[b], L.chunk_v, L.N_pad, L.chunk_v * 2, kBlockK, kBlockM);
-    ok &= make_map(&gm[b].b[0], W_s, L.d_s, L.V, L.d_s * 2, 64, 64);
-    // dW_s: A = G^T (MN-major), B = compacted h_s (hi part) as K x N (MN-major)
-    ok &= make_map(&gm[b].a[1], gbuf[b], L.chunk_v, L.N_pad, L.chunk_v * 2, 64, 64);
-    ok &= make_map(&gm[b].b[1], w.hs, L.d_s, L.N_pad, L.lda_s * 2, 64, 64);
-  }
+  // one gradient-chunk buffer: per chunk the sweep writes it and the GEMMs then read it, in stream
+  // order (two tensor-bound kernels gain nothing from overlapping; serial launches measured faster)
+  SweepMaps maps;
+  GemmMaps gm;
+  bool ok = sweep_maps(L, w, W_s, W_t, maps);
+  // gradient chunk written by the sweep epilogue: bf16 32 x 32 boxes, 64-byte rows
+  ok &= make_map(&maps.g_out, w.G, L.chunk_v, L.N_pad, L.chunk_v * 2, 32, 32, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
+                 CU_TENSOR_MAP_SWIZZLE_64B);
+  ok &= make_out_map(&gm.out[0], w.dhc, L.d_s, L.N_pad);
+  ok &= make_out_map(&gm.out[1], dW_s, L.d_s, L.V);
+  // dh_s: A = G (K-major, box 64 x 128), B = W_s chunk as K x N (MN-major, 64 x 64 boxes)
+  ok &= make_map(&gm.a[0], w.G, L.chunk_v, L.N_pad, L.chunk_v * 2, kBlockK, kBlockM);
+  ok &= make_map(&gm.b[0], W_s, L.d_s, L.V, L.d_s * 2, 64, 64);
+  // dW_s: A = G^T (MN-major), B = compacted h_s (hi part) as K x N (MN-major)
+  ok &= make_map(&gm.a[1], w.G, L.chunk_v, L.N_pad, L.chunk_v * 2, 64, 64);
+  ok &= make_map(&gm.b[1], w.hs, L.d_s, L.N_pad, L.lda_s * 2, 64, 64);
   if (!ok) return NB_ERR_CUDA;
 
   SweepArgs a = base_sweep_args(L, w, beta, tau);
   a.ldG = L.chunk_v;
   a.tiles_per_unit = 1;
+  a.n_big = 0;
+  a.G = w.G;
   GemmArgs g;
   std::memset(&g, 0, sizeof(g));
   g.nprob = 2;
@@ -813,29 +802,14 @@ nb_status nb_kl_backward(const nb_kl_shape* shape, const void* h_s, const void* 
 
   const int n_tt_max = int(L.N_pad / kPairM);
   const int n_dt = int((L.d_s + gemm_tile_n(g.wide) - 1) / gemm_tile_n(g.wide));   // output column tiles
-  AuxStream* ax = nullptr;
-  if ((s = aux_stream(&ax)) != NB_OK) return s;
-  // fork: the GEMMs run on a second stream, ordered after everything before this call
-  if (cudaEventRecord(ax->fork, st) != cudaSuccess || cudaStreamWaitEvent(ax->aux, ax->fork, 0) != cudaSuccess)
-    return NB_ERR_CUDA;
-  bool enq = true;
-  for (int c = 0; c < L.n_chunks && enq; ++c) {
-    const int b = c & 1;
+  for (int c = 0; c < L.n_chunks; ++c) {
     const int64_t v0 = int64_t(c) * L.chunk_v, v1 = std::min(L.V, v0 + L.chunk_v);
-    // buffer b was last read by the GEMMs of chunk c - 2
-    if (c >= 2 && cudaStreamWaitEvent(st, ax->used[b], 0) != cudaSuccess) { enq = false; break; }
     a.v_begin = int(v0);
     a.v_end = int(v1);
-    a.G = gbuf[b];
     a.sched = w.sched + 2 * c;
-    if (beta == 0.f) launch_sweep<kGradFkl>(dev, L, maps[b], a, st);
-    else if (beta == 1.f) launch_sweep<kGradRkl>(dev, L, maps[b], a, st);
-    else launch_sweep<kGradJsd>(dev, L, maps[b], a, st);
-    if (cudaEventRecord(ax->swept[b], st) != cudaSuccess ||
-        cudaStreamWaitEvent(ax->aux, ax->swept[b], 0) != cudaSuccess) {
-      enq = false;
-      break;
-    }
+    if (beta == 0.f) launch_sweep<kGradFkl>(dev, L, maps, a, st);
+    else if (beta == 1.f) launch_sweep<kGradRkl>(dev, L, maps, a, st);
+    else launch_sweep<kGradJsd>(dev, L, maps, a, st);
     dh.K = int(v1 - v0);
     dh.b_koff = int(v0);
     dh.accumulate = c > 0 ? 1 : 0;
@@ -844,15 +818,10 @@ nb_status nb_kl_backward(const nb_kl_shape* shape, const void* h_s, const void* 
     g.sched = w.sched + 2 * c + 1;
     const int tiles = n_tt_max * n_dt + int((v1 - v0 + kPairM - 1) / kPairM) * n_dt;
     next_cat(NB_KL_KERNEL_GEMM_BWD);
-    launch(gemm_kernel, dim3(pair_grid(dev, tiles)), dim3(kThreads), size_t(kSmemBytes), ax->aux, gm[b], g);
-    if (cudaEventRecord(ax->used[b], ax->aux) != cudaSuccess) enq = false;
+    launch(gemm_kernel, dim3(pair_grid(dev, tiles)), dim3(kThreads), size_t(kSmemBytes), st, gm, g);
   }
-  if (enq) launch(scatter_rows_kernel, dim3(unsigned(L.N_pad)), dim3(128), 0, ax->aux, (const float*)w.dhc,
-                  int(L.d_s), dh_s, (const int*)w.idx, (const Ctrl*)w.ctrl);
-  // join (also after a failure part-way): work after this call on `st` sees every GEMM result
-  if (cudaEventRecord(ax->join, ax->aux) != cudaSuccess || cudaStreamWaitEvent(st, ax->join, 0) != cudaSuccess)
-    return NB_ERR_CUDA;
-  if (!enq) return NB_ERR_CUDA;
+  launch(scatter_rows_kernel, dim3(unsigned(L.N_pad)), dim3(128), 0, st, (const float*)w.dhc, int(L.d_s), dh_s,
+         (const int*)w.idx, (const Ctrl*)w.ctrl);
   return check_launch();
 }
 
@@ -869,6 +838,13 @@ nb_status nb_kl_forward_noalloc(const nb_kl_shape* shape, const void* h_s, const
   if (s != NB_OK) return s;
   return nb_kl_forward(shape, h_s, W_s, h_t, W_t, labels, beta, tau, loss_tok, lse_s, lse_t, aux, loss_mean,
                        n_valid, ws, size_t(NB_KL_NOALLOC_SCRATCH_BYTES), stream);
+}
+
+nb_status nb_kl_noalloc_device_status(void* stream) {
+  void* ws = nullptr;
+  const nb_status s = fixed_scratch(&ws);
+  if (s != NB_OK) return s;
+  return nb_kl_device_status(ws, stream);
 }
 
 nb_status nb_kl_gram(const void* X, int64_t rows, int64_t d, float* G, void* workspace, void* stream) {
@@ -946,6 +922,20 @@ nb_status nb_kl_project(const void* X, int64_t rows, int64_t d, const void* B, i
   const int tiles = int((rows + kPairM - 1) / kPairM * ((k + gemm_tile_n(g.wide) - 1) / gemm_tile_n(g.wide)));
   next_cat(NB_KL_KERNEL_GEMM_PROJ);
   launch(gemm_kernel, dim3(pair_grid(dev, tiles)), dim3(kThreads), size_t(kSmemBytes), st, gm, g);
+  return check_launch();
+}
+
+nb_status nb_kl_spectral_select(const double* evals, const double* evecs, int64_t d, int64_t k, void* V_k,
+                                double* sigma, double* V_k_f64, void* stream) {
+  g_launches = 0;
+  if (!evals || !evecs || !V_k || !sigma) return NB_ERR_INVALID_ARG;
+  if (d < 1 || d > 65536 || k < 1 || k > d) return NB_ERR_INVALID_ARG;
+  DevInfo dev;
+  nb_status s = device_info(dev);
+  if (s != NB_OK) return s;
+  next_cat(NB_KL_KERNEL_GEMM_PROJ);
+  launch(spectral_select_kernel, dim3(unsigned(d)), dim3(256), 0, static_cast<cudaStream_t>(stream), evals, evecs,
+         int(d), int(k), static_cast<__nv_bfloat16*>(V_k), V_k_f64, sigma);
   return check_launch();
 }
 

@@ -408,6 +408,46 @@ __global__ void zero_masked_rows_kernel(const int64_t* __restrict__ labels, long
   for (int c = threadIdx.x; c < d; c += blockDim.x) row[c] = 0.f;
 }
 
+// ------------------------------------------------------------------ spectral basis selection
+// "Nitrobrew tweet analysis", thread item 6/8 and the "SVD-Nitrobrew" row of the evaluation
+// table: the teacher code keeps the k right singular vectors of W_t with the largest singular
+// values. Given the eigenpairs of G = W_t^T W_t (eigenvalue lambda_i = sigma_i^2, eigenvector i
+// in column i of the row-major [d, d] `evecs`, in any order), block i ranks eigenvalue i among
+// all d (larger first; equal values by index; NaN last) and, when its rank r is below k, copies
+// column i into column r of the basis: V_k (bf16, rounded to nearest even from fp64 once),
+// optionally the fp64 copy, and sigma_r = sqrt(max(lambda_i, 0)) (NaN for a NaN eigenvalue).
+__device__ __forceinline__ double rank_key(double x) { return isnan(x) ? -INFINITY : x; }
+
+__global__ void __launch_bounds__(256)
+    spectral_select_kernel(const double* __restrict__ evals, const double* __restrict__ evecs, int d, int k,
+                           __nv_bfloat16* __restrict__ Vk, double* __restrict__ Vk64, double* __restrict__ sigma) {
+  __shared__ int part[256];
+  const int i = blockIdx.x;
+  const double li = rank_key(evals[i]);
+  int cnt = 0;
+  for (int j = threadIdx.x; j < d; j += 256) {
+    const double lj = rank_key(evals[j]);
+    cnt += (lj > li || (lj == li && j < i)) ? 1 : 0;
+  }
+  part[threadIdx.x] = cnt;
+  __syncthreads();
+  for (int o = 128; o > 0; o >>= 1) {
+    if (threadIdx.x < o) part[threadIdx.x] += part[threadIdx.x + o];
+    __syncthreads();
+  }
+  const int r = part[0];
+  if (r >= k) return;
+  if (threadIdx.x == 0) {
+    const double l = evals[i];
+    sigma[r] = isnan(l) ? l : sqrt(l > 0.0 ? l : 0.0);   // a NaN eigenvalue stays NaN
+  }
+  for (int a = threadIdx.x; a < d; a += 256) {
+    const double v = evecs[(long long)a * d + i];
+    Vk[(long long)a * k + r] = __double2bfloat16(v);
+    if (Vk64) Vk64[(long long)a * k + r] = v;
+  }
+}
+
 // Test hook: wait on an mbarrier that nothing arrives at, with the given limit.
 __global__ void wait_timeout_kernel(int* status, unsigned long long limit_ns) {
   __shared__ uint64_t bar;

@@ -15,7 +15,8 @@
 // last read, normally long before the next tile's first-model phase ends).
 //
 // Warp roles (384 threads per CTA, one CTA per SM, persistent over work units):
-//   warp 0     TMA producer (both CTAs): 128 x 64 h tile + 128 x 64 W tile per stage, 6 stages
+//   warp 0     TMA producer (both CTAs): 128 x 64 h tile + 128 x 64 W tile per stage, 7 stages
+//              (6 in the gradient sweep, whose epilogue stages its output in the 7th)
 //   warp 1     MMA issuer (leader CTA only): 4 x tcgen05.mma 256x256x16 per K block; TMEM owner
 //   warps 2-3  idle (warpgroup 0 hands its registers to the epilogue: 56 vs 224 per thread)
 //   warps 4-11 epilogue: two warps per TMEM lane quarter, each thread one token row and one
@@ -26,8 +27,9 @@
 // arrive on the leader's tempty[]. Work ids come from the leader's TMA thread through a ring
 // mirrored into the peer CTA.
 //
-// A work unit is (256-row token tile, run of `tiles_per_unit` vocabulary tiles); each thread
-// writes its row's partial state once per unit (split = 2 * unit + column half).
+// A work unit is (256-row token tile, run of vocabulary tiles: `tiles_per_unit` of them for the
+// first `n_big` vocabulary units, one for the rest); each thread writes its row's partial state
+// once per unit (split = 2 * vocabulary unit + column half).
 #pragma once
 
 #include "common.cuh"
@@ -35,11 +37,10 @@
 namespace nbkl {
 
 struct SweepSmem {
-  uint8_t* a;           // kStages x 16 KB (wide GEMM tiles: a and b together as 4 x 48 KB)
-  uint8_t* b;           // kStages x 16 KB
-  uint8_t* out;         // kEpiWarps x 4 KB TMA-store staging
-  uint64_t* full;       // kStages (leader: TMA bytes of both CTAs)
-  uint64_t* empty;      // kStages (both: MMA commit)
+  uint8_t* a;           // operand stages: kMaxStages x (A 16 KB, B 16 KB); wide GEMM tiles 4 x 48 KB
+  uint8_t* out;         // kEpiWarps x 4 KB TMA-store staging (over the 7th stage; 6-stage kernels only)
+  uint64_t* full;       // kMaxStages (leader: TMA bytes of both CTAs)
+  uint64_t* empty;      // kMaxStages (both: MMA commit)
   uint64_t* tfull;      // sweep: [1] first model, [0] whole tile complete; GEMM: one per stage
   uint64_t* tempty;     // leader: accumulator released by all 16 epilogue warps of the pair
   uint64_t* drain;      // 1
@@ -53,23 +54,30 @@ __device__ __forceinline__ SweepSmem carve_smem(uint8_t* raw) {
   SweepSmem s;
   uint8_t* base = align1024(raw);
   s.a = base;
-  s.b = base + kStages * kATileBytes;
   s.out = base + kStages * kStageBytes;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(s.out + kEpiWarps * kStageOutBytes);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(base + kMaxStages * kStageBytes);
   s.full = bars;
-  s.empty = bars + kStages;
-  s.tfull = bars + 2 * kStages;
-  s.tempty = bars + 2 * kStages + 2;
-  s.drain = bars + 2 * kStages + 4;
-  s.ring_full = bars + 2 * kStages + 5;
+  s.empty = bars + kMaxStages;
+  s.tfull = bars + 2 * kMaxStages;
+  s.tempty = bars + 2 * kMaxStages + 2;
+  s.drain = bars + 2 * kMaxStages + 4;
+  s.ring_full = bars + 2 * kMaxStages + 5;
   s.ring_empty = s.ring_full + kRing;
   s.ring_slot = reinterpret_cast<int*>(s.ring_empty + kRing);
   s.tmem_slot = reinterpret_cast<uint32_t*>(s.ring_slot + kRing);
   return s;
 }
 
+// Operand tiles of narrow stage `st`.
+__device__ __forceinline__ uint32_t stage_a_addr(const SweepSmem& s, int st) {
+  return smem_addr(s.a + st * kStageBytes);
+}
+__device__ __forceinline__ uint32_t stage_b_addr(const SweepSmem& s, int st) {
+  return smem_addr(s.a + st * kStageBytes + kATileBytes);
+}
+
 __device__ __forceinline__ void init_barriers(const SweepSmem& s) {
-  for (int i = 0; i < kStages; ++i) {
+  for (int i = 0; i < kMaxStages; ++i) {
     mbar_init(&s.full[i], 1);
     mbar_init(&s.empty[i], 1);
   }
@@ -122,14 +130,24 @@ struct UnitGrid {
   int n_valid, n_tt, n_vt, n_vu, n_units;
 };
 
+// Vocabulary units: the first n_big units are runs of tiles_per_unit tiles, the rest single tiles
+// (n_big * tiles_per_unit <= n_vt), so the last work items of a launch are short.
 __device__ __forceinline__ UnitGrid unit_grid(const SweepArgs& p) {
   UnitGrid g;
   g.n_valid = *p.n_valid;
   g.n_tt = (g.n_valid + kPairM - 1) / kPairM;
   g.n_vt = (p.v_end - p.v_begin + kBlockN - 1) / kBlockN;
-  g.n_vu = (g.n_vt + p.tiles_per_unit - 1) / p.tiles_per_unit;
+  g.n_vu = p.n_big + (g.n_vt - p.n_big * p.tiles_per_unit);
   g.n_units = g.n_tt * g.n_vu;
   return g;
+}
+
+// First and one-past-last vocabulary tile of vocabulary unit vu.
+__device__ __forceinline__ int unit_t0(const SweepArgs& p, int vu) {
+  return vu < p.n_big ? vu * p.tiles_per_unit : p.n_big * p.tiles_per_unit + (vu - p.n_big);
+}
+__device__ __forceinline__ int unit_t1(const SweepArgs& p, int vu) {
+  return vu < p.n_big ? (vu + 1) * p.tiles_per_unit : unit_t0(p, vu) + 1;
 }
 
 // ------------------------------------------------------------------ work distribution
@@ -166,11 +184,12 @@ __device__ __forceinline__ bool ring_get(const SweepSmem& s, int it, int& id, co
 
 // Bounded wait for the copies a failed producer may still have in flight (leader: its full[]
 // barriers count the bytes of both CTAs).
+// `pend_*` hold the stage and parity of the last `n_stages` loads, at index (load number) % n_stages.
 __device__ __forceinline__ void drain_loads(const SweepSmem& s, const uint32_t* pend_stage,
-                                            const uint32_t* pend_par, int n_issued, int n_stages = kStages) {
+                                            const uint32_t* pend_par, int n_issued, int n_stages) {
   const int n = min(n_issued, n_stages);
   for (int i = 0; i < n; ++i) {
-    const int j = (n_issued - 1 - i) % kStages;
+    const int j = (n_issued - 1 - i) % n_stages;
     const uint32_t a = smem_addr(&s.full[pend_stage[j]]);
     const uint64_t t0 = global_timer_ns();
     while (!mbar_test(a, pend_par[j]) && global_timer_ns() - t0 < 100000000ull) {
@@ -196,11 +215,12 @@ __device__ __forceinline__ void release_accumulator(uint64_t* bar) {
 }
 
 // ------------------------------------------------------------------ producer (both CTAs)
+template <int NST>
 __device__ __forceinline__ void sweep_producer(const SweepMaps& maps, const SweepArgs& p, const UnitGrid& g,
                                                const SweepSmem& s, const WaitCtl& w, uint32_t rank) {
   int stage = 0;
   uint32_t phase = 0;
-  uint32_t pend_stage[kStages], pend_par[kStages];
+  uint32_t pend_stage[NST], pend_par[NST];
   int n_issued = 0;
   // first model = teacher when teacher_first
   const CUtensorMap* a1 = p.teacher_first ? &maps.a_t : &maps.a_s;
@@ -223,8 +243,8 @@ __device__ __forceinline__ void sweep_producer(const SweepMaps& maps, const Swee
     if (u < 0) break;
     const int vu = u / g.n_tt, tt = u % g.n_tt;
     const int row0 = tt * kPairM + int(rank) * kBlockM;
-    const int t_end = min((vu + 1) * p.tiles_per_unit, g.n_vt);
-    for (int t = vu * p.tiles_per_unit; t < t_end && ok; ++t) {
+    const int t_end = unit_t1(p, vu);
+    for (int t = unit_t0(p, vu); t < t_end && ok; ++t) {
       const int v0 = p.v_begin + t * kBlockN + int(rank) * kHalfB;
       for (int kb = 0; kb < nk1 + nk2; ++kb) {
         if (!mbar_wait_cl(&s.empty[stage], phase ^ 1u, w)) { ok = false; break; }
@@ -233,19 +253,20 @@ __device__ __forceinline__ void sweep_producer(const SweepMaps& maps, const Swee
         const int kbb = k % (one ? bm1 : bm2);
         const uint32_t bar = smem_addr(&s.full[stage]);
         if (rank == 0) mbar_arrive_expect_tx(&s.full[stage], kPairStageBytes);
-        tma_load_2d_pair(smem_addr(s.a + stage * kATileBytes), one ? a1 : a2, bar, k * kBlockK, row0);
-        tma_load_2d_pair(smem_addr(s.b + stage * kBTileBytes), one ? b1 : b2, bar, kbb * kBlockK, v0);
-        pend_stage[n_issued % kStages] = stage;
-        pend_par[n_issued % kStages] = phase;
+        tma_load_2d_pair(stage_a_addr(s, stage), one ? a1 : a2, bar, k * kBlockK, row0);
+        tma_load_2d_pair(stage_b_addr(s, stage), one ? b1 : b2, bar, kbb * kBlockK, v0);
+        pend_stage[n_issued % NST] = stage;
+        pend_par[n_issued % NST] = phase;
         ++n_issued;
-        if (++stage == kStages) { stage = 0; phase ^= 1u; }
+        if (++stage == NST) { stage = 0; phase ^= 1u; }
       }
     }
   }
-  if (!ok && rank == 0) drain_loads(s, pend_stage, pend_par, n_issued);
+  if (!ok && rank == 0) drain_loads(s, pend_stage, pend_par, n_issued, NST);
 }
 
 // ------------------------------------------------------------------ MMA issuer (leader)
+template <int NST>
 __device__ __forceinline__ void sweep_mma(const SweepArgs& p, const UnitGrid& g, const SweepSmem& s,
                                           uint32_t tmem_base, const WaitCtl& w) {
   int stage = 0;
@@ -258,8 +279,8 @@ __device__ __forceinline__ void sweep_mma(const SweepArgs& p, const UnitGrid& g,
     if (!ring_get(s, it, u, w, false)) { ok = false; break; }
     if (u < 0) break;
     const int vu = u / g.n_tt;
-    const int t_end = min((vu + 1) * p.tiles_per_unit, g.n_vt);
-    for (int t = vu * p.tiles_per_unit; t < t_end && ok; ++t, ++lt) {
+    const int t_end = unit_t1(p, vu);
+    for (int t = unit_t0(p, vu); t < t_end && ok; ++t, ++lt) {
       for (int kb = 0; kb < nk1 + nk2; ++kb) {
         const bool one = kb < nk1;
         const int k = one ? kb : kb - nk1;
@@ -271,15 +292,15 @@ __device__ __forceinline__ void sweep_mma(const SweepArgs& p, const UnitGrid& g,
         // TMA bytes are ordered by the barrier's transaction count: no tcgen05 fence here
         if (!mbar_wait(&s.full[stage], phase, w)) { ok = false; break; }
         const uint32_t d = tmem_base + (one ? 0 : kBlockN);
-        const uint32_t sa = smem_addr(s.a + stage * kATileBytes);
-        const uint32_t sb = smem_addr(s.b + stage * kBTileBytes);
+        const uint32_t sa = stage_a_addr(s, stage);
+        const uint32_t sb = stage_b_addr(s, stage);
 #pragma unroll
         for (int j = 0; j < kBlockK / 16; ++j) {
           umma_bf16_pair(d, make_sdesc(sa + j * 32, 16, 1024), make_sdesc(sb + j * 32, 16, 1024), kIdescKK,
                          (k > 0 || j > 0) ? 1u : 0u);
         }
         umma_commit_pair_both(smem_addr(&s.empty[stage]));
-        if (++stage == kStages) { stage = 0; phase ^= 1u; }
+        if (++stage == NST) { stage = 0; phase ^= 1u; }
         // first accumulator complete: the epilogues copy it out while the second model runs
         if (kb == nk1 - 1) umma_commit_pair_both(smem_addr(&s.tfull[1]));
       }
@@ -516,8 +537,8 @@ __device__ __forceinline__ void sweep_epilogue(const SweepMaps& maps, const Swee
     float* const lab_dst = (MODE <= kStateT && p.side) ? p.label_x + row : nullptr;
     RowState r{kNegBig, 0.f, kNegBig, 0.f, 0.f, 0.f};
     float js = 0.f, ks = 0.f;
-    const int t_end = min((vu + 1) * p.tiles_per_unit, g.n_vt);
-    for (int t = vu * p.tiles_per_unit; t < t_end; ++t, ++lt) {
+    const int t_end = unit_t1(p, vu);
+    for (int t = unit_t0(p, vu); t < t_end; ++t, ++lt) {
       const int v0 = p.v_begin + t * kBlockN + half * kHalfN;
       if (!mbar_wait_cl(&s.tfull[1], lt & 1u, w)) return;   // first model complete
       tc_fence_after();
@@ -588,10 +609,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   const UnitGrid g = unit_grid(p);
   const WaitCtl w{p.status, p.wait_limit_ns};
 
+  // the gradient sweep stages its output tiles, the state and JSD sweeps take a 7th operand stage
+  constexpr int NST = MODE >= kGradFkl ? kStages : kMaxStages;
   if (warp < kEpiWarp0) {
     regs_shrink<kRegsCtl>();
-    if (warp == 0 && lane == 0) sweep_producer(maps, p, g, s, w, rank);
-    if (warp == 1 && lane == 0 && rank == 0) sweep_mma(p, g, s, tmem_base, w);
+    if (warp == 0 && lane == 0) sweep_producer<NST>(maps, p, g, s, w, rank);
+    if (warp == 1 && lane == 0 && rank == 0) sweep_mma<NST>(p, g, s, tmem_base, w);
   } else {
     regs_grow<kRegsEpi>();
     sweep_epilogue<MODE>(maps, p, g, s, tmem_base, w);

@@ -6,9 +6,10 @@ With the thin SVD ``W_t = U S V^T`` and ``V_k`` the right singular vectors of th
 singular values:
 
 * once per teacher checkpoint, :func:`spectral_factor`: the Gram matrix ``W_t^T W_t`` on the
-  library's tcgen05 GEMM (``nb_kl_gram``), its eigenvectors (a d_t x d_t symmetric
+  library's tcgen05 GEMM (``nb_kl_gram``), its eigenpairs (a d_t x d_t symmetric
   eigendecomposition, ``torch.linalg.eigh`` in float64: the one library step, off the
-  per-step path), ``V_k`` rounded to bf16, and ``W_t' = W_t V_k`` (``nb_kl_project``);
+  per-step path), the k largest and their ``V_k`` rounded to bf16 (``nb_kl_spectral_select``),
+  and ``W_t' = W_t V_k`` (``nb_kl_project``);
 * every step, on the teacher's side, :func:`teacher_code`: ``h_t' = h_t V_k``
   (``nb_kl_project``), k values per token instead of d_t;
 * the loss then runs unchanged on ``(h_t', W_t')`` with d_t = k.
@@ -74,6 +75,23 @@ class SpectralBasis:
     V_k_f64: torch.Tensor    # [d_t, k] float64 eigenvectors before rounding
 
 
+def select_basis(evals: torch.Tensor, evecs: torch.Tensor, k: int):
+    """(V_k bf16 [d, k], sigma float64 [k], V_k float64 [d, k]) from the eigenpairs of W_t^T W_t
+    (``nb_kl_spectral_select``: the k largest eigenvalues, their eigenvectors rounded to bf16
+    once, sigma = sqrt(max(lambda, 0)))."""
+    d = evals.shape[0]
+    for name, t, shp in (("evals", evals, (d,)), ("evecs", evecs, (d, d))):
+        if not t.is_cuda or t.dtype != torch.float64 or tuple(t.shape) != shp or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous float64 CUDA tensor of shape {shp}")
+    V_k = torch.empty((d, k), dtype=torch.bfloat16, device=evals.device)
+    V64 = torch.empty((d, k), dtype=torch.float64, device=evals.device)
+    sigma = torch.empty((k,), dtype=torch.float64, device=evals.device)
+    code = _abi.lib().nb_kl_spectral_select(evals.data_ptr(), evecs.data_ptr(), d, k, V_k.data_ptr(),
+                                            sigma.data_ptr(), V64.data_ptr(), _stream_ptr(evals.device))
+    _abi.check("nb_kl_spectral_select", code)
+    return V_k, sigma, V64
+
+
 def spectral_factor(W_t: torch.Tensor, k: int) -> SpectralBasis:
     """Rank-k spectral basis of the teacher unembedding W_t [V, d_t] (bf16)."""
     _check_bf16("W_t", W_t)
@@ -81,11 +99,8 @@ def spectral_factor(W_t: torch.Tensor, k: int) -> SpectralBasis:
     if not 8 <= k <= d_t or k % 8:
         raise ValueError("k must be a multiple of 8 in [8, d_t]")
     G = gram(W_t).double()
-    evals, evecs = torch.linalg.eigh(G)                # ascending
-    order = torch.argsort(evals, descending=True)[:k]
-    V64 = evecs[:, order].contiguous()
-    sigma = evals[order].clamp_min(0).sqrt()
-    V_k = V64.to(torch.bfloat16).contiguous()
+    evals, evecs = torch.linalg.eigh(G)                # the one library step: a d_t x d_t solver
+    V_k, sigma, V64 = select_basis(evals.contiguous(), evecs.contiguous(), k)
     return SpectralBasis(V_k=V_k, W_code=project(W_t, V_k), sigma=sigma, V_k_f64=V64)
 
 

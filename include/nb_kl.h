@@ -189,6 +189,17 @@ NB_KL_API nb_status nb_kl_gram(const void* X, int64_t rows, int64_t d, float* G,
 NB_KL_API nb_status nb_kl_project(const void* X, int64_t rows, int64_t d, const void* B, int64_t k, void* Y,
                         void* workspace, void* stream);
 
+/* Rank-k basis from the eigenpairs of G = W_t^T W_t ("Nitrobrew tweet analysis", thread item 6/8
+ * and the evaluation table's "SVD-Nitrobrew" row: the code keeps the right singular vectors of
+ * the k largest singular values of W_t). evals [d] fp64 and evecs [d, d] fp64 row-major with
+ * eigenvector i in column i (the layout of a symmetric eigensolver's output; any eigenvalue
+ * order). Writes V_k [d, k] bf16 row-major: column r is the eigenvector of the r-th largest
+ * eigenvalue (ties by index, NaN last), rounded to nearest even from fp64 once; sigma [k] fp64:
+ * sqrt(max(lambda, 0)), the singular values of W_t (NaN stays NaN); and, unless NULL, V_k_f64 [d, k] fp64, the
+ * same columns unrounded. 1 <= k <= d <= 65536; all buffers on the device, caller-owned. */
+NB_KL_API nb_status nb_kl_spectral_select(const double* evals, const double* evecs, int64_t d, int64_t k,
+                                          void* V_k, double* sigma, double* V_k_f64, void* stream);
+
 /* ---- Teacher -> student hand-off of hidden states -----------------------------------------
  * "Nitrobrew tweet analysis", thread items 3/8 and 4/8 and section "OPD 为什么更痛": when teacher
  * and student sit on different GPUs, what must cross to the loss is the teacher's final hidden
@@ -238,6 +249,14 @@ NB_KL_API nb_status nb_kl_forward_noalloc(const nb_kl_shape* shape, const void* 
                                           const void* h_t, const void* W_t, const int64_t* labels, float beta,
                                           float tau, float* loss_tok, float* lse_s, float* lse_t, float* aux,
                                           float* loss_mean, int64_t* n_valid, void* stream);
+
+/* Device status word of nb_kl_forward_noalloc's fixed scratch on the current device, read the
+ * way nb_kl_device_status reads a caller's workspace: synchronises `stream`, then returns NB_OK,
+ * or NB_ERR_TIMEOUT when a bounded pipeline wait of the last call ran out (its outputs are then
+ * not valid), or NB_ERR_CUDA. Like every other use of the shared array, call it after the
+ * forward it checks and before the next nb_kl_forward_noalloc on this device: the next call
+ * clears the word. The pages have no counterpart. */
+NB_KL_API nb_status nb_kl_noalloc_device_status(void* stream);
 
 /* Static text for a status code. */
 NB_KL_API const char* nb_kl_status_string(nb_status status);

@@ -169,10 +169,10 @@ def test_spectral_argument_errors(L):
 
 def test_chunk_columns(L):
     lib = L.lib()
-    # default: ~8192 gradient tiles of 128 x 256 per launch, at least 4 d_s, in [2048, 32768]
-    assert lib.nb_kl_chunk_columns(L.shape_ptr(shape(L))) == 32768
+    # default: ~16384 gradient tiles of 128 x 256 per launch, at least 4 d_s, in [2048, 65536]
+    assert lib.nb_kl_chunk_columns(L.shape_ptr(shape(L))) == 65536
     assert lib.nb_kl_chunk_columns(L.shape_ptr(shape(L, N=32768, ds=4096, dt=512))) == 16384
-    assert lib.nb_kl_chunk_columns(L.shape_ptr(shape(L, N=65536, ds=256, dt=256))) == 4096
+    assert lib.nb_kl_chunk_columns(L.shape_ptr(shape(L, N=65536, ds=256, dt=256))) == 8192
     assert lib.nb_kl_chunk_columns(L.shape_ptr(shape(L, N=256, V=1000, ds=256, dt=256))) == 1024
     # an explicit chunk is kept; an invalid shape gives 0
     assert lib.nb_kl_chunk_columns(L.shape_ptr(shape(L, chunk=4096))) == 4096

@@ -72,6 +72,36 @@ def test_project(rows, d, k):
     assert not bad.any(), f"{bad.sum()} elements off"
 
 
+def _f64_to_bf16_bits(x):
+    """bf16 bit patterns of float64 values rounded to nearest even in one step (normal range)."""
+    b = np.ascontiguousarray(x, dtype=np.float64).view(np.uint64)
+    lsb = (b >> np.uint64(45)) & np.uint64(1)
+    r = (b + np.uint64((1 << 44) - 1) + lsb) & ~np.uint64((1 << 45) - 1)
+    return (r.view(np.float64).astype(np.float32).view(np.uint32) >> np.uint32(16)).astype(np.uint16)
+
+
+@pytest.mark.parametrize("d,k", [(200, 40), (64, 64), (1, 1), (520, 8)])
+def test_select_basis_exact(d, k):
+    """nb_kl_spectral_select against a plain host selection: the k largest eigenvalues (ties by
+    index, NaN last), their eigenvector columns exactly, bf16 by one rounding, sqrt(max(l, 0))."""
+    import torch
+    from full_vocab_kl_b200 import spectral
+    rng = np.random.default_rng(d * 1000 + k)
+    evals = rng.standard_normal(d) * 5.0
+    if d >= 8:
+        evals[3] = evals[5]                  # a tie
+        evals[6] = np.nan
+        evals[7] = -abs(evals[7])            # negative: sigma clamps to 0
+    evecs = rng.standard_normal((d, d))
+    V_k, sigma, V64 = spectral.select_basis(torch.from_numpy(evals).cuda(), torch.from_numpy(evecs).cuda(), k)
+    torch.cuda.synchronize()
+    key = np.where(np.isnan(evals), -np.inf, evals)
+    order = sorted(range(d), key=lambda i: (-key[i], i))[:k]
+    np.testing.assert_array_equal(V64.cpu().numpy(), evecs[:, order])
+    np.testing.assert_array_equal(_host(V_k), _f64_to_bf16_bits(evecs[:, order]))
+    np.testing.assert_array_equal(sigma.cpu().numpy(), np.sqrt(np.maximum(evals[order], 0.0)))   # NaN stays NaN
+
+
 def test_factor_matches_oracle_svd():
     from full_vocab_kl_b200 import spectral
     V, d, k = 20000, 256, 64

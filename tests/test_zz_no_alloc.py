@@ -35,6 +35,9 @@ def _noalloc(x):
         out["n_valid"].data_ptr(), ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
     _abi.check("nb_kl_forward_noalloc", code)
     torch.cuda.synchronize()
+    # the fixed scratch's status word: no bounded wait of this call ran out
+    assert _abi.lib().nb_kl_noalloc_device_status(
+        ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)) == _abi.NB_OK
     got = {k: out[k].cpu().numpy().astype(np.float64) for k in ("loss_tok", "lse_s", "lse_t", "aux")}
     got["loss_mean"] = float(out["loss_mean"].item())
     got["n_valid"] = int(out["n_valid"].item())
@@ -61,7 +64,9 @@ def test_noalloc_rejects_shapes_beyond_the_fixed_scratch():
     shape = _abi.Shape(n_tokens=65536, vocab=151936, d_s=4096, d_t=4096, h_dtype=0, reserved=0,
                        ignore_index=-100, chunk_v=0)
     assert _abi.lib().nb_kl_workspace_size(_abi.shape_ptr(shape), 1.0) > _abi.NOALLOC_SCRATCH_BYTES
-    fake = [ctypes.c_void_p(0x10000 * (i + 1)) for i in range(11)]
-    code = _abi.lib().nb_kl_forward_noalloc(_abi.shape_ptr(shape), *fake[:5], 1.0, 1.0, *fake[5:11],
+    # null pointers: the size check answers before any pointer is used, and if it ever did not,
+    # the pointer checks would refuse the call before a launch
+    null = [None] * 11
+    code = _abi.lib().nb_kl_forward_noalloc(_abi.shape_ptr(shape), *null[:5], 1.0, 1.0, *null[5:11],
                                             ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
     assert code == _abi.NB_ERR_WORKSPACE
