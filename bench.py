@@ -59,6 +59,53 @@ def measured_peaks():
     return dict(FALLBACK), "fallback"
 
 
+# SM clock of the sustained cuBLAS measurement when the peaks file does not record it (the
+# median under load of the pool's sustained run) and the boost clock of the part
+SUSTAINED_MHZ_DEFAULT = 1275.0
+MAX_MHZ_DEFAULT = 1965.0
+
+
+def _flat(d, prefix=""):
+    for k, v in (d.items() if isinstance(d, dict) else []):
+        key = f"{prefix}.{k}" if prefix else str(k)
+        if isinstance(v, dict):
+            yield from _flat(v, key)
+        else:
+            yield key.lower(), v
+
+
+def peak_clocks(peaks):
+    """(burst MHz, sustained MHz) of the peak measurements, from the peaks file's clock fields
+    where it records them (a key naming a clock and the run), else the defaults."""
+    burst, sustained = None, None
+    for k, v in _flat(peaks):
+        if not isinstance(v, (int, float)) or not ("mhz" in k or "clock" in k):
+            continue
+        if "sustained" in k and ("median" in k or sustained is None):
+            sustained = float(v)
+        elif "burst" in k and burst is None:
+            burst = float(v)
+    return burst, sustained if sustained is not None else SUSTAINED_MHZ_DEFAULT
+
+
+def choose_peak(peaks, src, run_mhz, max_mhz):
+    """The dense bf16 peak that applies at the clock the timed run held: the burst figure when
+    the run's median SM clock under load is within 5% of the burst measurement's clock (the
+    part's maximum when that is not recorded), the sustained figure when it is within 5% of the
+    sustained measurement's clock, else the burst figure scaled by the clock ratio."""
+    burst = float(peaks.get("bf16_tflops", FALLBACK["bf16_tflops"]))
+    sustained = float(peaks.get("bf16_tflops_sustained", FALLBACK["bf16_tflops_sustained"]))
+    b_mhz, s_mhz = peak_clocks(peaks)
+    b_mhz = b_mhz or max_mhz or MAX_MHZ_DEFAULT
+    if not run_mhz:
+        return burst, f"{src} bf16_tflops (burst; no clock record for this run)", b_mhz
+    if run_mhz >= 0.95 * b_mhz:
+        return burst, f"{src} bf16_tflops (burst, measured near {b_mhz:.0f} MHz)", b_mhz
+    if abs(run_mhz - s_mhz) <= 0.05 * s_mhz:
+        return sustained, f"{src} bf16_tflops_sustained (measured near {s_mhz:.0f} MHz)", s_mhz
+    return burst * run_mhz / b_mhz, f"{src} bf16_tflops x {run_mhz:.0f} / {b_mhz:.0f} MHz (burst at the run's clock)", run_mhz
+
+
 def algorithmic_flops(w, n_valid, V=None, proj=0.0):
     """FLOPs of the method on valid rows: forward sweep, [JSD second sweep], recompute sweep,
     dh_s and dW_s products (V: the vocabulary rows this rank holds), and the teacher-code
@@ -137,7 +184,7 @@ class ClockSampler:
             self.f = open(self.path, "w")
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "100"], stdout=self.f, stderr=subprocess.DEVNULL)
+                 "-lms", "20"], stdout=self.f, stderr=subprocess.DEVNULL)
             time.sleep(0.3)
         except (OSError, FileNotFoundError):
             self.proc = None
@@ -275,6 +322,71 @@ def workload_config(w, n_valid, world):
             "l2": "inputs larger than L2 (unembeddings >= 1 GB per step), no flush"}
 
 
+# ----------------------------------------------------------------------------- other workloads
+EXTRA_WORKLOADS = ("long_jsd", "large_vocab", "spectral")
+
+
+def measure_workload(name, steps, warmup, dev, gpu_index):
+    """Device-timed forward + backward of one more workload with its inputs resident, timed with
+    CUDA events on the launching stream and with its own clock record (one GPU)."""
+    import torch
+
+    import full_vocab_kl_b200 as nb
+    from synthetic import make_inputs
+    x = make_inputs(name)
+    w = x.workload
+    nv = int((x.labels != -100).sum())
+
+    def to_dev(a):
+        if a.dtype == np.uint16:
+            return torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(dev)
+        return torch.from_numpy(a).to(dev)
+
+    h_s, h_t, W_s, W_t = (to_dev(getattr(x, k)) for k in ("h_s", "h_t", "W_s", "W_t"))
+    labels = torch.from_numpy(x.labels).to(dev)
+    N = labels.shape[0]
+    f32 = dict(dtype=torch.float32, device=dev)
+    shape = nb.make_shape(h_s, W_s, h_t, W_t, labels)
+    ws = torch.empty(nb.workspace_bytes(shape, w.beta), dtype=torch.uint8, device=dev)
+    out = {"loss_tok": torch.empty(N, **f32), "lse_s": torch.empty(N, **f32), "lse_t": torch.empty(N, **f32),
+           "aux": torch.empty(N, **f32), "loss_mean": torch.empty((), **f32),
+           "n_valid": torch.empty((), dtype=torch.int64, device=dev)}
+    dh = torch.empty((N, w.d_s), **f32)
+    dW = (torch.from_numpy(x.dW_init).to(dev) if w.accumulate_dW else torch.empty((w.V, w.d_s), **f32))
+    go = torch.ones((), **f32)
+
+    def step():
+        nb.kl_forward(h_s, W_s, h_t, W_t, labels, w.beta, w.tau, workspace=ws, out=out)
+        nb.kl_backward(h_s, W_s, h_t, W_t, labels, w.beta, w.tau, out["lse_s"], out["lse_t"], out["aux"], go,
+                       dh_s=dh, dW_s=dW, accumulate_dW=w.accumulate_dW, workspace=ws)
+
+    stream = torch.cuda.current_stream(dev)
+    for _ in range(warmup):
+        step()
+    clocks = ClockSampler(gpu_index)
+    clocks.start()
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    clk = clocks.stop()
+    status = nb.device_status(ws)
+    ms = e0.elapsed_time(e1) / steps
+    flops = sum(algorithmic_flops(w, nv).values())
+    tflops = flops / (ms * 1e-3) / 1e12
+    res = {"workload": name, "tokens": N, "valid_tokens": nv, "vocab": w.V, "d_s": w.d_s, "d_t": w.d_t,
+           "beta": w.beta, "tau": w.tau, "accumulate_dW": w.accumulate_dW, "steps": steps, "warmup": warmup,
+           "ms_per_step": ms, "tokens_per_s": N / (ms * 1e-3), "tflops": tflops,
+           "pct_bf16_peak_datasheet": 100.0 * tflops / DATASHEET_BF16_TFLOPS,
+           "device_status": int(status), "clocks": clk}
+    del h_s, h_t, W_s, W_t, ws, dW, dh
+    torch.cuda.empty_cache()
+    return res
+
+
 # ----------------------------------------------------------------------------- library arm
 def run_library(args):
     import torch
@@ -388,7 +500,10 @@ def run_library(args):
     dh = torch.empty((N, w.d_s), **f32)
     dW = torch.zeros((V_rank, w.d_s), **f32) if w.accumulate_dW else torch.empty((V_rank, w.d_s), **f32)
 
-    def step(hs, ht, lab):
+    def step(hs, ht, lab, marks=None):
+        """One forward + backward; with `marks`, events on the launching stream bracket the
+        backward call (its kernels, including any on the library's second stream, which the
+        call joins back before it returns)."""
         if args.vocab_parallel:
             CountingKernels.launches = 0
             f = vp_forward(hs, W_s, ht, W_t, lab, w.beta, w.tau, vocab_offset=v0, side=args.side, kernels=kern,
@@ -408,8 +523,13 @@ def run_library(args):
         nb.kl_forward(hs, W_s, ht, W_t, lab, w.beta, w.tau, workspace=ws, out=out, chunk_v=args.chunk_v,
                       side=args.side)
         n1 = lib.nb_kl_last_launch_count()
+        if marks is not None:
+            marks.append((torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)))
+            marks[-1][0].record(stream)
         nb.kl_backward(hs, W_s, ht, W_t, lab, w.beta, w.tau, out["lse_s"], out["lse_t"], out["aux"], grad_out,
                        dh_s=dh, dW_s=dW, accumulate_dW=w.accumulate_dW, workspace=ws, chunk_v=args.chunk_v)
+        if marks is not None:
+            marks[-1][1].record(stream)
         return n0 + n1 + lib.nb_kl_last_launch_count()
 
     stream = torch.cuda.current_stream(dev)
@@ -418,11 +538,10 @@ def run_library(args):
     mem0 = torch.cuda.memory_allocated(dev)
     torch.cuda.reset_peak_memory_stats(dev)
 
-    # ---- device-timed region
+    # ---- device-timed region (the headline): the library's per-launch timing hook is off
     clocks = ClockSampler(local)
     if rank == 0:
         clocks.start()
-    lib.nb_kl_timing_enable(1)
     barrier()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
@@ -431,14 +550,33 @@ def run_library(args):
         launches += step(h_s, h_t, labels)
     e1.record(stream)
     barrier()
+    clk = clocks.stop() if rank == 0 else None
+    ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
+    peak_extra = torch.cuda.max_memory_allocated(dev) - mem0
+
+    # ---- per-kernel pass, after the headline and not part of it: the same number of steps
+    # with the library's per-launch events on (each launch bracketed on its own stream) and
+    # every backward call bracketed on the launching stream
+    clocks_k = ClockSampler(local)
+    if rank == 0:
+        clocks_k.start()
+    lib.nb_kl_timing_enable(1)
+    barrier()
+    marks = []
+    ek0, ek1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ek0.record(stream)
+    for _ in range(args.steps):
+        step(h_s, h_t, labels, marks=None if args.vocab_parallel else marks)
+    ek1.record(stream)
+    barrier()
     lib.nb_kl_timing_enable(0)
+    clk_k = clocks_k.stop() if rank == 0 else None
     ncat = len(_abi.KERNEL_CATEGORIES)
     ms_arr = (ctypes.c_double * ncat)()
     cnt_arr = (ctypes.c_int * ncat)()
     lib.nb_kl_timing_read(ctypes.cast(ms_arr, ctypes.c_void_p), ctypes.cast(cnt_arr, ctypes.c_void_p), ncat)
-    clk = clocks.stop() if rank == 0 else None
-    ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
-    peak_extra = torch.cuda.max_memory_allocated(dev) - mem0
+    ms_kpass = ek0.elapsed_time(ek1) / args.steps
+    bwd_ms = (sum(a.elapsed_time(b) for a, b in marks) / len(marks)) if marks else None
 
     # ---- end-to-end through the public API with host buffers: every step copies its inputs
     # from pinned host memory and reads its loss back; the copy of step i + 1's inputs runs on
@@ -504,7 +642,18 @@ def run_library(args):
         per_launch_ms = kms[dom] / max(kcount[dom], 1)
         per_launch_flops = flops[dom] / max(kcount[dom], 1)
         achieved = per_launch_flops / (per_launch_ms * 1e-3) / 1e12
-        peak = peaks.get("bf16_tflops_sustained", FALLBACK["bf16_tflops_sustained"])
+        run_mhz = (clk_k or {}).get("sm_mhz") or (clk or {}).get("sm_mhz")
+        max_mhz = (clk or {}).get("sm_max_mhz")
+        peak, peak_desc, peak_mhz = choose_peak(peaks, peak_src, run_mhz, max_mhz)
+        step_peak, step_peak_desc, _ = choose_peak(peaks, peak_src, (clk or {}).get("sm_mhz"), max_mhz)
+        # the backward as one unit: gradient sweeps and GEMMs over the backward call's span
+        bwd_unit = None
+        if bwd_ms:
+            bwd_flops = flops["sweep_grad"] + flops["gemm_bwd"]
+            bwd_unit = {"ms": bwd_ms, "flops": bwd_flops, "tflops": bwd_flops / (bwd_ms * 1e-3) / 1e12,
+                        "frac": bwd_flops / (bwd_ms * 1e-3) / 1e12 / peak,
+                        "note": "gradient sweeps + dh_s/dW_s GEMMs (+ the call's row kernels) between events "
+                                "bracketing each backward call on the launching stream"}
         chunk_cols = lib.nb_kl_chunk_columns(_abi.shape_ptr(shape))
         traffic = (profiled_traffic(dom, w.name, chunk_cols)
                    if not (args.vocab_parallel or args.front_end) else None)
@@ -523,11 +672,15 @@ def run_library(args):
             "tflops": tflops, "pct_bf16_peak_datasheet": 100.0 * tflops / DATASHEET_BF16_TFLOPS,
             "model_tflops": model_flops(w, n_valid, V_rank) * world / (ms_step * 1e-3) / 1e12,
             "pct_bf16_peak_measured": 100.0 * tflops / peaks.get("bf16_tflops", FALLBACK["bf16_tflops"]),
+            "pct_bf16_peak_at_run_clock": 100.0 * tflops / step_peak, "step_peak_source": step_peak_desc,
             "roofline": {"bound": "tensor", "kernel": dom, "achieved": achieved, "peak": peak,
-                         "peak_source": f"{peak_src} bf16_tflops_sustained", "unit": "TFLOP/s",
-                         "frac": achieved / peak, "traffic": traffic,
-                         "algorithmic_flops_per_launch": per_launch_flops, "launch_ms": per_launch_ms},
+                         "peak_source": peak_desc, "peak_clock_mhz": peak_mhz, "run_sm_mhz": run_mhz,
+                         "unit": "TFLOP/s", "frac": achieved / peak, "traffic": traffic,
+                         "algorithmic_flops_per_launch": per_launch_flops, "launch_ms": per_launch_ms,
+                         "timed_in": "per-kernel pass after the headline (same steps, per-launch events on)"},
+            "backward_unit": bwd_unit,
             "kernel_ms_per_step": kms, "kernel_launches_per_step": kcount,
+            "kernel_pass": {"ms_per_step": ms_kpass, "kernel_ms_sum": sum(kms.values()), "clocks": clk_k},
             "kernel_tflops": {c: (flops[c] / (kms[c] * 1e-3) / 1e12 if kms[c] > 0 else None)
                               for c in ("sweep_fwd", "sweep_jsd", "sweep_grad", "gemm_bwd", "gemm_proj")},
             "e2e": {"value": units / (ms_e2e / e2e_steps * 1e-3), "unit": "tokens/s",
@@ -544,6 +697,14 @@ def run_library(args):
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
+    plain = not (args.vocab_parallel or args.front_end or args.handoff or args.side)
+    if rank == 0 and world == 1 and plain and args.workload == DEFAULT_WORKLOAD and not args.no_workloads:
+        # the other workloads of the method's configuration list, each timed on its own
+        del ws, dW, dh, W_s, W_t
+        torch.cuda.empty_cache()
+        wl = [measure_workload(n, args.workload_steps, args.warmup, dev, local) for n in EXTRA_WORKLOADS]
+        result["workloads"] = wl
+        result["workloads_weakest"] = min(wl, key=lambda r: r["tflops"])["workload"]
     if rank == 0 and not args.no_cpu_baseline and not args.front_end:
         result["cpu_baseline"] = cpu_baseline(x)
     if rank == 0:
@@ -561,6 +722,9 @@ def main():
     ap.add_argument("--impl", default="library", choices=["library", "reference"])
     ap.add_argument("--chunk-v", type=int, default=0, help="backward vocabulary chunk (0: library default)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-workloads", action="store_true",
+                    help="skip the device-timed lines of the other workloads (long_jsd, large_vocab, spectral)")
+    ap.add_argument("--workload-steps", type=int, default=10, help="timed steps of each other workload")
     ap.add_argument("--side", action="store_true",
                     help="forward with the student entropy / sampled-token log-prob side outputs")
     ap.add_argument("--vocab-parallel", action="store_true",

@@ -86,3 +86,25 @@ def test_flop_counts():
     jsd = WORKLOADS["long_jsd"]
     fj = bench.algorithmic_flops(jsd, 6144)
     assert fj["sweep_jsd"] == fj["sweep_fwd"] > 0
+
+
+def test_peak_follows_the_run_clock():
+    """The roofline's peak is the burst figure when the run held its clock near the burst
+    measurement's, the sustained figure near the sustained measurement's clock, and the burst
+    figure scaled by the clock ratio in between."""
+    import bench
+    peaks = {"bf16_tflops": 1630.0, "bf16_tflops_sustained": 1371.8}
+    p, desc, mhz = bench.choose_peak(peaks, "measured", 1942.0, 1965.0)
+    assert p == 1630.0 and "burst" in desc and mhz == 1965.0
+    p, desc, mhz = bench.choose_peak(peaks, "measured", 1290.0, 1965.0)
+    assert p == 1371.8 and "sustained" in desc and mhz == bench.SUSTAINED_MHZ_DEFAULT
+    p, desc, mhz = bench.choose_peak(peaks, "measured", 1620.0, 1965.0)
+    assert p == pytest.approx(1630.0 * 1620.0 / 1965.0) and mhz == 1620.0
+    # clock fields recorded in the peaks file take precedence over the defaults
+    rec = dict(peaks, clocks={"bf16_burst_sm_mhz": 1900.0, "bf16_sustained_sm_mhz_median": 1400.0})
+    assert bench.peak_clocks(rec) == (1900.0, 1400.0)
+    assert bench.choose_peak(rec, "measured", 1410.0, 1965.0)[0] == 1371.8
+    assert bench.choose_peak(rec, "measured", 1850.0, 1965.0)[0] == 1630.0
+    # no clock record: the burst figure, said so
+    p, desc, _ = bench.choose_peak(peaks, "measured", None, None)
+    assert p == 1630.0 and "no clock record" in desc
