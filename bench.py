@@ -151,22 +151,29 @@ def kernel_source_sha():
     return h.hexdigest()[:16]
 
 
-def profiled_traffic(kernel: str, workload: str, chunk_v: int):
-    """Per-launch DRAM bytes (read + write) of `kernel` from the committed full-size ncu summary
-    of the workload, if that summary was taken from the current device code with the same
-    backward chunk (the per-launch traffic of the backward kernels scales with it)."""
-    p = os.path.join(ROOT, "profiles", f"fullsize_{workload}.md")
+# profiling-size workload with the same token shape as a bench workload (its ncu summaries carry the
+# per-launch DRAM bytes of each kernel)
+PROFILE_OF = {"opd_0p6b_4b": "opd_0p6b_4b_v24k_prof"}
+
+
+def profiled_traffic(kernel: str, workload: str, columns_per_launch: float):
+    """DRAM bytes (read + write) of one launch of `kernel`, from the committed ncu summary of the
+    workload's profiling-size twin (same tokens, smaller vocabulary), scaled by the vocabulary
+    columns one launch covers: the unembedding rows, the gradient chunk and the dW_s rows grow in
+    proportion to them. None unless that summary was taken from the current device code."""
+    prof = PROFILE_OF.get(workload)
+    if prof is None:
+        return None
+    p = os.path.join(ROOT, "profiles", f"{kernel}_{prof}.md")
     if not os.path.exists(p):
         return None
     txt = open(p).read()
     m_sha = re.search(r"kernel_source_sha:\s*([0-9a-f]+)", txt)
-    m_tr = re.search(re.escape(kernel) + r"\.dram_bytes_per_launch:\s*([0-9.eE+]+)", txt)
-    m_ch = re.search(r"chunk_columns:\s*([0-9]+)", txt)
-    if not m_sha or not m_tr or m_sha.group(1) != kernel_source_sha():
+    m_b = re.search(r"dram_bytes_per_launch:\s*([0-9.eE+]+)", txt)
+    m_c = re.search(r"profiled_vocab_columns_per_launch:\s*([0-9]+)", txt)
+    if not (m_sha and m_b and m_c) or m_sha.group(1) != kernel_source_sha():
         return None
-    if not m_ch or int(m_ch.group(1)) != chunk_v:
-        return None
-    return float(m_tr.group(1))
+    return float(m_b.group(1)) * columns_per_launch / float(m_c.group(1))
 
 
 class ClockSampler:
@@ -655,7 +662,8 @@ def run_library(args):
                         "note": "gradient sweeps + dh_s/dW_s GEMMs (+ the call's row kernels) between events "
                                 "bracketing each backward call on the launching stream"}
         chunk_cols = lib.nb_kl_chunk_columns(_abi.shape_ptr(shape))
-        traffic = (profiled_traffic(dom, w.name, chunk_cols)
+        cols_per_launch = V_rank / max(kcount[dom], 1) if dom != "gemm_proj" else 0.0
+        traffic = (profiled_traffic(dom, w.name, cols_per_launch)
                    if not (args.vocab_parallel or args.front_end) else None)
         config = workload_config(w, n_valid, world)
         if args.vocab_parallel:
@@ -677,6 +685,8 @@ def run_library(args):
                          "peak_source": peak_desc, "peak_clock_mhz": peak_mhz, "run_sm_mhz": run_mhz,
                          "unit": "TFLOP/s", "frac": achieved / peak, "traffic": traffic,
                          "algorithmic_flops_per_launch": per_launch_flops, "launch_ms": per_launch_ms,
+                         "traffic_source": ("ncu DRAM bytes of the profiling-size twin workload, scaled by the "
+                                            "vocabulary columns per launch") if traffic else None,
                          "timed_in": "per-kernel pass after the headline (same steps, per-launch events on)"},
             "backward_unit": bwd_unit,
             "kernel_ms_per_step": kms, "kernel_launches_per_step": kcount,

@@ -108,6 +108,14 @@ PROFILE_WORKLOADS = {
         "opd_0p6b_4b_prof", 1, 640, 1024, 2560, 75776, 1.0, 1.0, 3.0,
         teacher="correlated", mask="prefix", masked_per_seq=128,
         description="profiling size of opd_0p6b_4b: 640 tokens (512 valid), V 75776"),
+    # the OPD workload's token shape (4 x 2048 tokens, 819-token prompt prefix masked per
+    # sequence, 4916 valid) with a 24576-row vocabulary: the backward's GEMM launch keeps the
+    # full workload's proportions (dh_s: 20 x 2 tiles over the chunk, dW_s: 96 x 2 tiles over
+    # the valid tokens) in under 1 GB on the device; the unembeddings (176 MB) exceed L2
+    "opd_0p6b_4b_v24k_prof": Workload(
+        "opd_0p6b_4b_v24k_prof", 4, 2048, 1024, 2560, 24576, 1.0, 1.0, 3.0,
+        teacher="correlated", mask="prefix", masked_per_seq=819,
+        description="profiling size of opd_0p6b_4b: its 8192 tokens (4916 valid), V 24576"),
     "spectral_prof": Workload(
         "spectral_prof", 2, 4096, 4096, 512, 32768, 1.0, 1.0, 3.0,
         teacher="spectral", mask="random", masked_per_seq=1434,

@@ -108,3 +108,22 @@ def test_peak_follows_the_run_clock():
     # no clock record: the burst figure, said so
     p, desc, _ = bench.choose_peak(peaks, "measured", None, None)
     assert p == 1630.0 and "no clock record" in desc
+
+
+def test_profiled_traffic_scales_by_columns_and_checks_the_code_hash(tmp_path, monkeypatch):
+    """The roofline's traffic comes from the profiling-size twin's ncu summary, scaled by the
+    vocabulary columns one launch covers, and only while the summary matches the device code."""
+    import bench
+    prof = tmp_path / "profiles"
+    prof.mkdir()
+    (prof / "sweep_grad_opd_0p6b_4b_v24k_prof.md").write_text(
+        f"kernel_source_sha: {bench.kernel_source_sha()}\n"
+        "profiled_vocab_columns_per_launch: 24576\ndram_bytes_per_launch: 4.0e8\n")
+    real_sha = bench.kernel_source_sha()
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    monkeypatch.setattr(bench, "kernel_source_sha", lambda: real_sha)
+    assert bench.profiled_traffic("sweep_grad", "opd_0p6b_4b", 49152) == pytest.approx(8.0e8)
+    assert bench.profiled_traffic("sweep_grad", "long_jsd", 49152) is None        # no twin
+    assert bench.profiled_traffic("gemm_bwd", "opd_0p6b_4b", 49152) is None       # no summary
+    monkeypatch.setattr(bench, "kernel_source_sha", lambda: "0" * 16)              # code changed
+    assert bench.profiled_traffic("sweep_grad", "opd_0p6b_4b", 49152) is None
