@@ -292,6 +292,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     }
   }
   const uint32_t tmem_base = pair_prologue(s);
+  pdl_wait();
+  pdl_launch_dependents();
   const int nv = *p.n_valid;
   const WaitCtl w{p.status, p.wait_limit_ns};
   if (warp < kEpiWarp0) {

@@ -246,15 +246,28 @@ bool make_out_map(CUtensorMap* m, float* base, uint64_t cols, uint64_t rows) {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
 
-template <typename K, typename... Args>
-void launch(K kernel, dim3 grid, dim3 block, size_t smem, cudaStream_t st, Args... args) {
+// Every launch allows programmatic dependent launch: the kernel may start (and run its set-up)
+// while the previous kernel in the stream finishes; its first global-memory access waits for that
+// kernel (pdl_wait in every kernel). A failed launch is reported by check_launch().
+template <typename... KArgs, typename... Args>
+void launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, Args... args) {
   TimingRec r{g_cat, nullptr, nullptr};
   if (g_timing.on) {
     r.a = g_timing.get();
     r.b = g_timing.get();
     cudaEventRecord(r.a, st);
   }
-  kernel<<<grid, block, smem, st>>>(args...);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr;
+  attr.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr.val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = &attr;
+  cfg.numAttrs = 1;
+  cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
   ++g_launches;
   if (g_timing.on) {
     cudaEventRecord(r.b, st);
@@ -440,12 +453,13 @@ nb_status prepare(Prep& P, const nb_kl_shape* shape, const void* h_s, const void
   const Ws& w = P.w;
   // all-ones bits are a NaN: a label column the sweep never meets leaves a NaN log-probability
   if (side && cudaMemsetAsync(w.labx, 0xFF, size_t(L.N_pad) * 4, st) != cudaSuccess) return NB_ERR_CUDA;
+  // work counters zeroed first, so that the kernels of the call follow one another directly
+  if (cudaMemsetAsync(w.sched, 0, size_t(2 * L.n_chunks + 2) * 4, st) != cudaSuccess) return NB_ERR_CUDA;
   launch(compact_kernel, dim3(1), dim3(kScanThreads), 0, st, labels, int(L.N), (long long)shape->ignore_index,
          w.idx, w.ctrl, n_valid, (const float*)nullptr, tau, side ? w.rlab : (int*)nullptr, (long long)L.V,
          (long long)v_off);
   launch_gather(L, w, h_s, L.d_s, w.hs, L.lda_s, st);
   launch_gather(L, w, h_t, L.d_t, w.ht, L.lda_t, st);
-  if (cudaMemsetAsync(w.sched, 0, size_t(2 * L.n_chunks + 2) * 4, st) != cudaSuccess) return NB_ERR_CUDA;
   if (!sweep_maps(L, w, W_s, W_t, P.maps)) return NB_ERR_CUDA;
   P.a = base_sweep_args(L, w, beta, tau);
   P.a.out = w.state;
@@ -575,12 +589,12 @@ nb_status vp_jsd_partial_impl(const nb_kl_shape* shape, const void* h_s, const v
   P.w = carve(P.L, workspace);
   const Layout& L = P.L;
   const Ws& w = P.w;
+  if (cudaMemsetAsync(w.sched, 0, size_t(2 * L.n_chunks + 2) * 4, st) != cudaSuccess) return NB_ERR_CUDA;
   launch(compact_kernel, dim3(1), dim3(kScanThreads), 0, st, labels, int(L.N), (long long)shape->ignore_index,
          w.idx, w.ctrl, (int64_t*)nullptr, (const float*)nullptr, tau, (int*)nullptr, (long long)L.V, 0ll);
   // the global LSEs become the per-row base-2 constants of the second pass (aux is unused there)
   launch_gather(L, w, h_s, L.d_s, w.hs, L.lda_s, st, lse_s, lse_t, lse_s);
   launch_gather(L, w, h_t, L.d_t, w.ht, L.lda_t, st);
-  if (cudaMemsetAsync(w.sched, 0, size_t(2 * L.n_chunks + 2) * 4, st) != cudaSuccess) return NB_ERR_CUDA;
   if (!sweep_maps(L, w, W_s, W_t, P.maps)) return NB_ERR_CUDA;
   P.a = base_sweep_args(L, w, beta, tau);
   P.a.sched = w.sched;
@@ -748,6 +762,7 @@ nb_status nb_kl_backward(const nb_kl_shape* shape, const void* h_s, const void* 
     if (!accumulate_dW && cudaMemsetAsync(dW_s, 0, size_t(L.V) * L.d_s * 4, st) != cudaSuccess) return NB_ERR_CUDA;
     return NB_OK;
   }
+  if (cudaMemsetAsync(w.sched, 0, size_t(2 * L.n_chunks + 2) * 4, st) != cudaSuccess) return NB_ERR_CUDA;
   launch(compact_kernel, dim3(1), dim3(kScanThreads), 0, st, labels, int(L.N), (long long)shape->ignore_index,
          w.idx, w.ctrl, (int64_t*)nullptr, grad_out, tau, (int*)nullptr, (long long)L.V, 0ll);
   launch_gather(L, w, h_s, L.d_s, w.hs, L.lda_s, st, lse_s, lse_t, aux);
@@ -755,7 +770,6 @@ nb_status nb_kl_backward(const nb_kl_shape* shape, const void* h_s, const void* 
   launch(zero_masked_rows_kernel, dim3(unsigned(L.N)), dim3(128), 0, st, labels, (long long)shape->ignore_index,
          dh_s, int(L.d_s));
 
-  if (cudaMemsetAsync(w.sched, 0, size_t(2 * L.n_chunks + 2) * 4, st) != cudaSuccess) return NB_ERR_CUDA;
   // one gradient-chunk buffer: per chunk the sweep writes it and the GEMMs then read it, in stream
   // order (two tensor-bound kernels gain nothing from overlapping; serial launches measured faster)
   SweepMaps maps;

@@ -24,6 +24,16 @@ __device__ __forceinline__ uint64_t global_timer_ns() {
   return t;
 }
 
+// ------------------------------------------------------------------ programmatic dependent launch
+// Every kernel of the library is launched with programmatic stream serialization: it may be
+// scheduled while the previous kernel in the stream is still finishing, runs its set-up (barriers,
+// tensor memory, descriptor prefetch), and waits here before its first access to global memory
+// (read or write); the wait returns once the preceding grids have completed and their writes are
+// visible (at once for a launch without the attribute).
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+// Lets the next kernel in the stream be scheduled (it still waits in pdl_wait for this one).
+__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // ------------------------------------------------------------------ mbarrier
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count) : "memory");

@@ -28,6 +28,8 @@ __global__ void __launch_bounds__(kScanThreads) compact_kernel(const int64_t* __
                                                                const float* grad_out, float tau,
                                                                int* __restrict__ row_label, long long V,
                                                                long long v_off) {
+  pdl_wait();
+  pdl_launch_dependents();
   __shared__ int warp_sums[32];
   __shared__ int s_total;
   const int per = (N + kScanThreads - 1) / kScanThreads;
@@ -82,6 +84,8 @@ __global__ void gather_rows_kernel(const void* __restrict__ src, int d, __nv_bfl
                                    // optional per-row constants (backward): base-2 LSEs and aux
                                    const float* lse_s, const float* lse_t, const float* aux, float* row_l2s,
                                    float* row_l2t, float* row_aux) {
+  pdl_wait();
+  pdl_launch_dependents();
   const int i = blockIdx.x;
   const int nv = ctrl->n_valid;
   const int rows_needed = ((nv + kPairM - 1) / kPairM) * kPairM;
@@ -133,6 +137,8 @@ __global__ void __launch_bounds__(kMergeRows * kMergeLanes)
                  const Ctrl* __restrict__ ctrl, int kl_dir, float* loss_tok, float* lse_s, float* lse_t, float* aux,
                  float* row_l2s, float* row_l2t, int side, const float* __restrict__ label_x, float* entropy_s,
                  float* logp_label, float* vp_state, long long vp_ld) {
+  pdl_wait();
+  pdl_launch_dependents();
   __shared__ float sm_s[kMergeLanes][kMergeRows], sm_t[kMergeLanes][kMergeRows];
   __shared__ double sl_s[kMergeLanes][kMergeRows], sl_t[kMergeLanes][kMergeRows], sa[kMergeLanes][kMergeRows];
   __shared__ double se[kMergeLanes][kMergeRows];
@@ -216,6 +222,8 @@ __global__ void __launch_bounds__(kMergeRows * kMergeLanes)
 __global__ void __launch_bounds__(kMergeRows * kMergeLanes)
     jsd_finalize_kernel(const float* __restrict__ part, long long fs, int ld, int n_split,
                         const int* __restrict__ idx, const Ctrl* __restrict__ ctrl, float* loss_tok, float* aux) {
+  pdl_wait();
+  pdl_launch_dependents();
   __shared__ double sj[kMergeLanes][kMergeRows], sk[kMergeLanes][kMergeRows];
   const int r = threadIdx.x % kMergeRows, j = threadIdx.x / kMergeRows;
   const int nv = ctrl->n_valid;
@@ -255,6 +263,8 @@ __global__ void __launch_bounds__(128)
     vp_combine_kernel(const float* __restrict__ st, int n_parts, long long N, const int64_t* __restrict__ labels,
                       long long ignore_index, int kl_dir, float* loss_tok, float* lse_s, float* lse_t, float* aux,
                       float* entropy_s, float* logp_label) {
+  pdl_wait();
+  pdl_launch_dependents();
   const long long row = blockIdx.x * 128ll + threadIdx.x;
   if (row >= N) return;
   const long long P = (long long)kVpFields * N;   // elements per part
@@ -302,6 +312,8 @@ __global__ void __launch_bounds__(128)
 __global__ void __launch_bounds__(128)
     vp_jsd_combine_kernel(const float* __restrict__ parts, int n_parts, long long N,
                           const int64_t* __restrict__ labels, long long ignore_index, float* loss_tok, float* aux) {
+  pdl_wait();
+  pdl_launch_dependents();
   const long long row = blockIdx.x * 128ll + threadIdx.x;
   if (row >= N) return;
   double js = 0.0, ks = 0.0;
@@ -319,6 +331,8 @@ __global__ void __launch_bounds__(128)
 __global__ void __launch_bounds__(1024)
     mean_count_kernel(const float* __restrict__ loss_tok, const int64_t* __restrict__ labels, long long N,
                       long long ignore_index, float* loss_mean, int64_t* n_valid) {
+  pdl_wait();
+  pdl_launch_dependents();
   __shared__ double part[1024];
   __shared__ long long cnt[1024];
   double s = 0.0;
@@ -352,6 +366,8 @@ __global__ void __launch_bounds__(1024)
 __global__ void __launch_bounds__(256)
     handoff_rows_kernel(const uint4* __restrict__ src, uint4* __restrict__ dst, long long n_rows,
                         long long row_vecs, const int64_t* __restrict__ labels, long long ignore_index) {
+  pdl_wait();
+  pdl_launch_dependents();
   const long long warp_id = (blockIdx.x * 256ll + threadIdx.x) >> 5;
   const long long n_warps = (long long)gridDim.x * 8;
   const int lane = threadIdx.x & 31;
@@ -374,6 +390,8 @@ __global__ void __launch_bounds__(256)
 // Deterministic masked mean: fixed-order fp64 sum of loss_tok (masked rows hold 0).
 __global__ void __launch_bounds__(1024) mean_kernel(const float* __restrict__ loss_tok, int N,
                                                     const Ctrl* __restrict__ ctrl, float* loss_mean) {
+  pdl_wait();
+  pdl_launch_dependents();
   __shared__ double part[1024];
   double s = 0.0;
   for (int i = threadIdx.x; i < N; i += 1024) s += loss_tok[i];
@@ -392,6 +410,8 @@ __global__ void __launch_bounds__(1024) mean_kernel(const float* __restrict__ lo
 // dh_s[idx[i]] = dh_c[i] for the valid rows (the GEMMs accumulate into the compacted dh_c).
 __global__ void scatter_rows_kernel(const float* __restrict__ src, int d, float* __restrict__ dst,
                                     const int* __restrict__ idx, const Ctrl* __restrict__ ctrl) {
+  pdl_wait();
+  pdl_launch_dependents();
   const int i = blockIdx.x;
   if (i >= ctrl->n_valid) return;
   const float4* in = reinterpret_cast<const float4*>(src + (long long)i * d);
@@ -402,6 +422,8 @@ __global__ void scatter_rows_kernel(const float* __restrict__ src, int d, float*
 // Zero the dh_s rows of masked positions (valid rows are written by the scatter).
 __global__ void zero_masked_rows_kernel(const int64_t* __restrict__ labels, long long ignore_index, float* dh,
                                         int d) {
+  pdl_wait();
+  pdl_launch_dependents();
   const int r = blockIdx.x;
   if (labels[r] != ignore_index) return;
   float* row = dh + (long long)r * d;
@@ -421,6 +443,8 @@ __device__ __forceinline__ double rank_key(double x) { return isnan(x) ? -INFINI
 __global__ void __launch_bounds__(256)
     spectral_select_kernel(const double* __restrict__ evals, const double* __restrict__ evecs, int d, int k,
                            __nv_bfloat16* __restrict__ Vk, double* __restrict__ Vk64, double* __restrict__ sigma) {
+  pdl_wait();
+  pdl_launch_dependents();
   __shared__ int part[256];
   const int i = blockIdx.x;
   const double li = rank_key(evals[i]);
@@ -450,6 +474,8 @@ __global__ void __launch_bounds__(256)
 
 // Test hook: wait on an mbarrier that nothing arrives at, with the given limit.
 __global__ void wait_timeout_kernel(int* status, unsigned long long limit_ns) {
+  pdl_wait();
+  pdl_launch_dependents();
   __shared__ uint64_t bar;
   if (threadIdx.x == 0) {
     mbar_init(&bar, 1);

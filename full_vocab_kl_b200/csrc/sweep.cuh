@@ -606,6 +606,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     if (MODE >= kGradFkl) tma_prefetch_map(&maps.g_out);
   }
   const uint32_t tmem_base = pair_prologue(s);
+  pdl_wait();
+  pdl_launch_dependents();
   const UnitGrid g = unit_grid(p);
   const WaitCtl w{p.status, p.wait_limit_ns};
 
