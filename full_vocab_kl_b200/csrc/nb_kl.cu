@@ -37,6 +37,7 @@ constexpr int kTailItems = 160;   // single-tile work items at the end of a forw
 constexpr size_t kCtrlBytes = 256;
 
 thread_local int g_launches = 0;
+thread_local bool g_launch_failed = false;   // a launch of the current call was refused
 
 // Opt-in per-kernel timing: events recorded on the launching stream around each launch.
 struct TimingRec {
@@ -267,7 +268,7 @@ void launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaSt
   attr.val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = &attr;
   cfg.numAttrs = 1;
-  cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+  if (cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...) != cudaSuccess) g_launch_failed = true;
   ++g_launches;
   if (g_timing.on) {
     cudaEventRecord(r.b, st);
@@ -279,7 +280,11 @@ void launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaSt
 // the next launch belongs to category `c`
 void next_cat(int c) { g_cat = c; }
 
-nb_status check_launch() { return cudaGetLastError() == cudaSuccess ? NB_OK : NB_ERR_CUDA; }
+nb_status check_launch() {
+  const bool failed = g_launch_failed;
+  g_launch_failed = false;
+  return (cudaGetLastError() == cudaSuccess && !failed) ? NB_OK : NB_ERR_CUDA;
+}
 
 struct Ws {
   Ctrl* ctrl;
@@ -518,6 +523,7 @@ nb_status forward_impl(const nb_kl_shape* shape, const void* h_s, const void* W_
                        float* aux, float* loss_mean, int64_t* n_valid, float* entropy_s, float* logp_label,
                        void* workspace, size_t workspace_bytes, void* stream) {
   g_launches = 0;
+  g_launch_failed = false;
   Prep P;
   nb_status s = validate_common(shape, h_s, W_s, h_t, W_t, labels, beta, tau, workspace, workspace_bytes, P.L);
   if (s != NB_OK) return s;
@@ -552,6 +558,7 @@ nb_status vp_state_impl(const nb_kl_shape* shape, int64_t v_off, const void* h_s
                         const void* W_t, const int64_t* labels, float beta, float tau, float* state,
                         void* workspace, size_t workspace_bytes, cudaStream_t st) {
   g_launches = 0;
+  g_launch_failed = false;
   Prep P;
   nb_status s = validate_common(shape, h_s, W_s, h_t, W_t, labels, beta, tau, workspace, workspace_bytes, P.L);
   if (s != NB_OK) return s;
@@ -576,6 +583,7 @@ nb_status vp_jsd_partial_impl(const nb_kl_shape* shape, const void* h_s, const v
                               const float* lse_t, float* part, void* workspace, size_t workspace_bytes,
                               cudaStream_t st) {
   g_launches = 0;
+  g_launch_failed = false;
   Prep P;
   nb_status s = validate_common(shape, h_s, W_s, h_t, W_t, labels, beta, tau, workspace, workspace_bytes, P.L);
   if (s != NB_OK) return s;
@@ -695,6 +703,7 @@ nb_status nb_kl_vp_combine(int64_t n_tokens, int n_parts, const float* states, c
                            int64_t ignore_index, float beta, float* loss_tok, float* lse_s, float* lse_t, float* aux,
                            float* entropy_s, float* logp_label, float* loss_mean, int64_t* n_valid, void* stream) {
   g_launches = 0;
+  g_launch_failed = false;
   if (n_tokens < 0 || n_tokens > (int64_t(1) << 30) || n_parts < 1 || n_parts > 4096) return NB_ERR_INVALID_ARG;
   if (!(beta >= 0.f && beta <= 1.f)) return NB_ERR_INVALID_ARG;
   if (!loss_mean || !n_valid) return NB_ERR_INVALID_ARG;
@@ -726,6 +735,7 @@ nb_status nb_kl_vp_jsd_combine(int64_t n_tokens, int n_parts, const float* parts
                                int64_t ignore_index, float* loss_tok, float* aux, float* loss_mean, int64_t* n_valid,
                                void* stream) {
   g_launches = 0;
+  g_launch_failed = false;
   if (n_tokens < 0 || n_tokens > (int64_t(1) << 30) || n_parts < 1 || n_parts > 4096) return NB_ERR_INVALID_ARG;
   if (!loss_mean || !n_valid) return NB_ERR_INVALID_ARG;
   if (n_tokens > 0 && (!parts || !labels || !loss_tok || !aux)) return NB_ERR_INVALID_ARG;
@@ -747,6 +757,7 @@ nb_status nb_kl_backward(const nb_kl_shape* shape, const void* h_s, const void* 
                          const float* lse_t, const float* aux, const float* grad_out, float* dh_s, float* dW_s,
                          int accumulate_dW, void* workspace, size_t workspace_bytes, void* stream) {
   g_launches = 0;
+  g_launch_failed = false;
   Layout L;
   nb_status s = validate_common(shape, h_s, W_s, h_t, W_t, labels, beta, tau, workspace, workspace_bytes, L);
   if (s != NB_OK) return s;
@@ -844,6 +855,7 @@ nb_status nb_kl_forward_noalloc(const nb_kl_shape* shape, const void* h_s, const
                                 float* lse_s, float* lse_t, float* aux, float* loss_mean, int64_t* n_valid,
                                 void* stream) {
   g_launches = 0;
+  g_launch_failed = false;
   const size_t need = nb_kl_workspace_size(shape, beta);
   if (need == 0) return NB_ERR_INVALID_ARG;
   if (need > size_t(NB_KL_NOALLOC_SCRATCH_BYTES)) return NB_ERR_WORKSPACE;
@@ -863,6 +875,7 @@ nb_status nb_kl_noalloc_device_status(void* stream) {
 
 nb_status nb_kl_gram(const void* X, int64_t rows, int64_t d, float* G, void* workspace, void* stream) {
   g_launches = 0;
+  g_launch_failed = false;
   if (!X || !G || !workspace) return NB_ERR_INVALID_ARG;
   if (rows < 1 || d < 8 || d % 8 || rows > (int64_t(1) << 30) || d > 65536) return NB_ERR_INVALID_ARG;
   if (!aligned16(X) || !aligned16(G) || !aligned16(workspace)) return NB_ERR_INVALID_ARG;
@@ -901,6 +914,7 @@ nb_status nb_kl_gram(const void* X, int64_t rows, int64_t d, float* G, void* wor
 nb_status nb_kl_project(const void* X, int64_t rows, int64_t d, const void* B, int64_t k, void* Y, void* workspace,
                         void* stream) {
   g_launches = 0;
+  g_launch_failed = false;
   if (!X || !B || !Y || !workspace) return NB_ERR_INVALID_ARG;
   if (rows < 1 || d < 8 || k < 8 || d % 8 || k % 8) return NB_ERR_INVALID_ARG;
   if (rows > (int64_t(1) << 30) || d > 65536 || k > 65536) return NB_ERR_INVALID_ARG;
@@ -942,6 +956,7 @@ nb_status nb_kl_project(const void* X, int64_t rows, int64_t d, const void* B, i
 nb_status nb_kl_spectral_select(const double* evals, const double* evecs, int64_t d, int64_t k, void* V_k,
                                 double* sigma, double* V_k_f64, void* stream) {
   g_launches = 0;
+  g_launch_failed = false;
   if (!evals || !evecs || !V_k || !sigma) return NB_ERR_INVALID_ARG;
   if (d < 1 || d > 65536 || k < 1 || k > d) return NB_ERR_INVALID_ARG;
   DevInfo dev;
@@ -956,6 +971,7 @@ nb_status nb_kl_spectral_select(const double* evals, const double* evecs, int64_
 nb_status nb_kl_handoff_rows(const void* src, void* dst, int64_t n_rows, int64_t row_bytes, const int64_t* labels,
                              int64_t ignore_index, void* stream) {
   g_launches = 0;
+  g_launch_failed = false;
   if (n_rows < 0 || row_bytes < 16 || row_bytes % 16 || row_bytes > (int64_t(1) << 24)) return NB_ERR_INVALID_ARG;
   if (n_rows == 0) return NB_OK;
   if (!src || !dst || !aligned16(src) || !aligned16(dst)) return NB_ERR_INVALID_ARG;
@@ -989,6 +1005,7 @@ nb_status nb_kl_enable_peer_access(int peer_device) {
 nb_status nb_kl_debug_gemm(const void* A, int a_mn_major, const void* B, int b_mn_major, int64_t M, int64_t N,
                            int64_t K, float* C, void* workspace, void* stream) {
   g_launches = 0;
+  g_launch_failed = false;
   if (!A || !B || !C || !workspace) return NB_ERR_INVALID_ARG;
   if (M < 1 || N < 1 || K < 1 || M % 8 || N % 8 || K % 8) return NB_ERR_INVALID_ARG;
   if (M > (1 << 30) || N > (1 << 30) || K > (1 << 30)) return NB_ERR_INVALID_ARG;
@@ -1029,6 +1046,7 @@ nb_status nb_kl_debug_gemm(const void* A, int a_mn_major, const void* B, int b_m
 
 nb_status nb_kl_debug_wait_timeout(void* workspace, uint64_t limit_ns, void* stream) {
   g_launches = 0;
+  g_launch_failed = false;
   if (!workspace || !aligned16(workspace)) return NB_ERR_INVALID_ARG;
   if (limit_ns > 5000000000ull) return NB_ERR_INVALID_ARG;
   DevInfo dev;
