@@ -104,6 +104,8 @@ struct SweepArgs {
   int* sched;             // zeroed work counter: CTAs take units in order (null: static stride)
   int* status;
   unsigned long long wait_limit_ns;
+  int tt_group;           // token tiles per group of the work order (all vocabulary units of one
+                          // group before the next group)
 };
 
 // ------------------------------------------------------------------ backward GEMMs

@@ -35,6 +35,12 @@ constexpr unsigned long long kWaitLimitNs = 1000000000ull;  // 1 s per pipeline 
 constexpr int kTilesPerUnitFwd = 8;                          // 2048 vocabulary columns per unit
 constexpr int kTailItems = 160;   // single-tile work items at the end of a forward sweep (~2 waves of pairs)
 constexpr size_t kCtrlBytes = 256;
+// Compacted h rows of both models per token group of the sweeps' work order. Each of the B200's two
+// L2 halves keeps its own copy of lines its SMs read, so the rows re-read for every vocabulary tile
+// must fit in one half (~63 MB) beside the unembedding tiles in flight; measured best at 40 MB
+// (32-56 MB tried: 40 gave the shortest steps on the long-context, large-vocabulary and spectral
+// workloads; a workload whose rows fit in one group, like the OPD workload, is unaffected).
+constexpr double kTokenGroupBytes = 40.0 * 1024 * 1024;
 
 thread_local int g_launches = 0;
 thread_local bool g_launch_failed = false;   // a launch of the current call was refused
@@ -369,6 +375,9 @@ SweepArgs base_sweep_args(const Layout& L, const Ws& w, float beta, float tau) {
   a.gscale = &w.ctrl->gscale;
   a.status = &w.ctrl->status;
   a.wait_limit_ns = kWaitLimitNs;
+  // token tiles per group: the group's compacted rows of both models within kTokenGroupBytes
+  const double tile_bytes = double(kPairM) * double(L.lda_s + L.lda_t) * 2.0;
+  a.tt_group = int(std::min(double(1 << 30), std::max(1.0, std::floor(kTokenGroupBytes / tile_bytes))));
   return a;
 }
 

@@ -142,6 +142,25 @@ __device__ __forceinline__ UnitGrid unit_grid(const SweepArgs& p) {
   return g;
 }
 
+// Work order: token tiles in groups of tt_group; within a group, vocabulary-unit major (the
+// group's token tiles of one vocabulary unit are consecutive work items, so the pairs working at
+// the same time share the unembedding tiles), and a group's units all come before the next
+// group's (so the compacted rows re-read for every vocabulary tile stay few enough for L2).
+__device__ __forceinline__ void decode_unit(const SweepArgs& p, const UnitGrid& g, int u, int& vu, int& tt) {
+  const int G = p.tt_group;
+  const int n_full = g.n_tt / G;
+  const int per_group = G * g.n_vu;
+  if (u < n_full * per_group) {
+    const int grp = u / per_group, r = u % per_group;
+    vu = r / G;
+    tt = grp * G + r % G;
+  } else {
+    const int rem = g.n_tt - n_full * G, r = u - n_full * per_group;
+    vu = r / rem;
+    tt = n_full * G + r % rem;
+  }
+}
+
 // First and one-past-last vocabulary tile of vocabulary unit vu.
 __device__ __forceinline__ int unit_t0(const SweepArgs& p, int vu) {
   return vu < p.n_big ? vu * p.tiles_per_unit : p.n_big * p.tiles_per_unit + (vu - p.n_big);
@@ -241,7 +260,8 @@ __device__ __forceinline__ void sweep_producer(const SweepMaps& maps, const Swee
       break;
     }
     if (u < 0) break;
-    const int vu = u / g.n_tt, tt = u % g.n_tt;
+    int vu, tt;
+    decode_unit(p, g, u, vu, tt);
     const int row0 = tt * kPairM + int(rank) * kBlockM;
     const int t_end = unit_t1(p, vu);
     for (int t = unit_t0(p, vu); t < t_end && ok; ++t) {
@@ -278,7 +298,8 @@ __device__ __forceinline__ void sweep_mma(const SweepArgs& p, const UnitGrid& g,
     int u;
     if (!ring_get(s, it, u, w, false)) { ok = false; break; }
     if (u < 0) break;
-    const int vu = u / g.n_tt;
+    int vu, tt;
+    decode_unit(p, g, u, vu, tt);
     const int t_end = unit_t1(p, vu);
     for (int t = unit_t0(p, vu); t < t_end && ok; ++t, ++lt) {
       for (int kb = 0; kb < nk1 + nk2; ++kb) {
@@ -523,7 +544,8 @@ __device__ __forceinline__ void sweep_epilogue(const SweepMaps& maps, const Swee
     int u;
     if (!ring_get(s, it, u, w, true)) return;
     if (u < 0) break;
-    const int vu = u / g.n_tt, tt = u % g.n_tt;
+    int vu, tt;
+    decode_unit(p, g, u, vu, tt);
     const int row = tt * kPairM + int(rank) * kBlockM + row_in_tile;
     const bool row_ok = row < g.n_valid;
     if (MODE >= kJsd) {

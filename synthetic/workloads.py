@@ -116,6 +116,13 @@ PROFILE_WORKLOADS = {
         "opd_0p6b_4b_v24k_prof", 4, 2048, 1024, 2560, 24576, 1.0, 1.0, 3.0,
         teacher="correlated", mask="prefix", masked_per_seq=819,
         description="profiling size of opd_0p6b_4b: its 8192 tokens (4916 valid), V 24576"),
+    # the long_jsd workload's tokens, widths, mask and boosted rows with a 24576-row vocabulary
+    # (unembeddings 302 MB): its three sweeps (state, JSD pass, JSD gradient) at profiling size
+    "long_jsd_v24k_prof": Workload(
+        "long_jsd_v24k_prof", 1, 8192, 2048, 4096, 24576, 0.5, 2.0, 3.0,
+        teacher="correlated", mask="random", masked_per_seq=2048,
+        boost_frac=0.01, boost=20.0,
+        description="profiling size of long_jsd: its 8192 tokens (6144 valid), V 24576"),
     "spectral_prof": Workload(
         "spectral_prof", 2, 4096, 4096, 512, 32768, 1.0, 1.0, 3.0,
         teacher="spectral", mask="random", masked_per_seq=1434,

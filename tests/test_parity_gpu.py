@@ -32,6 +32,15 @@ def test_tiny_workload():
     full_check(make_inputs("tiny"))
 
 
+@pytest.mark.parametrize("beta", [1.0, 0.5])
+def test_token_groups_of_the_work_order(beta):
+    """Wide rows (d_s = d_t = 4096: 4 MB of compacted rows per 256-token tile) put the sweeps'
+    work order in groups of 10 token tiles: 5400 valid rows are 22 tiles, two full groups and a
+    remainder of 2; every row against the oracle, forward and backward (JSD: all three sweeps)."""
+    x = make_custom(5600, 4096, 4096, 1000, beta, 1.0, n_masked=200, teacher="independent")
+    full_check(x)
+
+
 @pytest.mark.parametrize("beta", [0.0, 1.0, 0.5, 0.3])
 def test_ragged_all_dims(beta):
     # 300 rows (tail of 44 rows), V 1000 (tail tile of 104 columns), K tails of 8 and 8
