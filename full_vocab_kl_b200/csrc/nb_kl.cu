@@ -80,7 +80,7 @@ struct Layout {
   int n_big;             // forward sweeps: vocabulary units of kTilesPerUnitFwd tiles (the rest are single tiles)
   int64_t chunk_v;
   int n_chunks;          // backward vocabulary chunks
-  size_t off_idx, off_hs, off_ht, off_rl2s, off_rl2t, off_raux, off_rlab, off_labx, off_sched, off_dhc, off_state,
+  size_t off_idx, off_inv, off_hs, off_ht, off_rl2s, off_rl2t, off_raux, off_rlab, off_labx, off_sched, off_dhc, off_state,
       off_part, off_G, g_bytes, total;
   long long fs_state;    // elements between state fields
 };
@@ -125,6 +125,7 @@ bool make_layout(const nb_kl_shape* sh, float beta, Layout& L) {
   const bool jsd = beta > 0.f && beta < 1.f;
   size_t off = kCtrlBytes;
   L.off_idx = off;   off = align256(off + size_t(L.N_pad) * 4);
+  L.off_inv = off;   off = align256(off + size_t(L.N_pad) * 4);   // compacted index of each position
   L.off_hs = off;    off = align256(off + size_t(L.N_pad) * L.lda_s * 2);
   L.off_ht = off;    off = align256(off + size_t(L.N_pad) * L.lda_t * 2);
   L.off_rl2s = off;  off = align256(off + size_t(L.N_pad) * 4);
@@ -295,6 +296,7 @@ nb_status check_launch() {
 struct Ws {
   Ctrl* ctrl;
   int* idx;
+  int* inv;
   int* sched;
   float* dhc;
   __nv_bfloat16 *hs, *ht;
@@ -309,6 +311,7 @@ Ws carve(const Layout& L, void* ws) {
   Ws w;
   w.ctrl = reinterpret_cast<Ctrl*>(b);
   w.idx = reinterpret_cast<int*>(b + L.off_idx);
+  w.inv = reinterpret_cast<int*>(b + L.off_inv);
   w.sched = reinterpret_cast<int*>(b + L.off_sched);
   w.dhc = reinterpret_cast<float*>(b + L.off_dhc);
   w.hs = reinterpret_cast<__nv_bfloat16*>(b + L.off_hs);
@@ -324,22 +327,26 @@ Ws carve(const Layout& L, void* ws) {
   return w;
 }
 
-void launch_gather(const Layout& L, const Ws& w, const void* h, int64_t d, __nv_bfloat16* dst, int64_t lda,
-                   cudaStream_t st, const float* lse_s = nullptr, const float* lse_t = nullptr,
-                   const float* aux = nullptr) {
-  const int half = int(lda / (L.split ? 2 : 1));
+// The valid rows of both hidden states into the compacted bf16 buffers (one launch); with lse_s,
+// also the per-row constants of the second pass and the backward.
+void launch_gathers(const Layout& L, const Ws& w, const void* h_s, const void* h_t, cudaStream_t st,
+                    const float* lse_s = nullptr, const float* lse_t = nullptr, const float* aux = nullptr) {
+  const int div = L.split ? 2 : 1;
+  const GatherSrc gs{h_s, int(L.d_s), int(L.lda_s), int(L.lda_s / div), w.hs};
+  const GatherSrc gt{h_t, int(L.d_t), int(L.lda_t), int(L.lda_t / div), w.ht};
   float *r2s = nullptr, *r2t = nullptr, *rax = nullptr;
   if (lse_s) {
     r2s = w.rl2s;
     r2t = w.rl2t;
     rax = w.raux;
   }
+  const dim3 grid(unsigned(L.N_pad), 2);
   if (L.split)
-    launch(gather_rows_kernel<true>, dim3(unsigned(L.N_pad)), dim3(128), 0, st, h, int(d), dst, int(lda), half,
-           (const int*)w.idx, (const Ctrl*)w.ctrl, lse_s, lse_t, aux, r2s, r2t, rax);
+    launch(gather_rows_kernel<true>, grid, dim3(128), 0, st, gs, gt, (const int*)w.idx, (const Ctrl*)w.ctrl, lse_s,
+           lse_t, aux, r2s, r2t, rax);
   else
-    launch(gather_rows_kernel<false>, dim3(unsigned(L.N_pad)), dim3(128), 0, st, h, int(d), dst, int(lda), half,
-           (const int*)w.idx, (const Ctrl*)w.ctrl, lse_s, lse_t, aux, r2s, r2t, rax);
+    launch(gather_rows_kernel<false>, grid, dim3(128), 0, st, gs, gt, (const int*)w.idx, (const Ctrl*)w.ctrl, lse_s,
+           lse_t, aux, r2s, r2t, rax);
 }
 
 bool sweep_maps(const Layout& L, const Ws& w, const void* W_s, const void* W_t, SweepMaps& m) {
@@ -471,9 +478,8 @@ nb_status prepare(Prep& P, const nb_kl_shape* shape, const void* h_s, const void
   if (cudaMemsetAsync(w.sched, 0, size_t(2 * L.n_chunks + 2) * 4, st) != cudaSuccess) return NB_ERR_CUDA;
   launch(compact_kernel, dim3(1), dim3(kScanThreads), 0, st, labels, int(L.N), (long long)shape->ignore_index,
          w.idx, w.ctrl, n_valid, (const float*)nullptr, tau, side ? w.rlab : (int*)nullptr, (long long)L.V,
-         (long long)v_off);
-  launch_gather(L, w, h_s, L.d_s, w.hs, L.lda_s, st);
-  launch_gather(L, w, h_t, L.d_t, w.ht, L.lda_t, st);
+         (long long)v_off, (int*)nullptr);
+  launch_gathers(L, w, h_s, h_t, st);
   if (!sweep_maps(L, w, W_s, W_t, P.maps)) return NB_ERR_CUDA;
   P.a = base_sweep_args(L, w, beta, tau);
   P.a.out = w.state;
@@ -608,10 +614,10 @@ nb_status vp_jsd_partial_impl(const nb_kl_shape* shape, const void* h_s, const v
   const Ws& w = P.w;
   if (cudaMemsetAsync(w.sched, 0, size_t(2 * L.n_chunks + 2) * 4, st) != cudaSuccess) return NB_ERR_CUDA;
   launch(compact_kernel, dim3(1), dim3(kScanThreads), 0, st, labels, int(L.N), (long long)shape->ignore_index,
-         w.idx, w.ctrl, (int64_t*)nullptr, (const float*)nullptr, tau, (int*)nullptr, (long long)L.V, 0ll);
+         w.idx, w.ctrl, (int64_t*)nullptr, (const float*)nullptr, tau, (int*)nullptr, (long long)L.V, 0ll,
+         (int*)nullptr);
   // the global LSEs become the per-row base-2 constants of the second pass (aux is unused there)
-  launch_gather(L, w, h_s, L.d_s, w.hs, L.lda_s, st, lse_s, lse_t, lse_s);
-  launch_gather(L, w, h_t, L.d_t, w.ht, L.lda_t, st);
+  launch_gathers(L, w, h_s, h_t, st, lse_s, lse_t, lse_s);
   if (!sweep_maps(L, w, W_s, W_t, P.maps)) return NB_ERR_CUDA;
   P.a = base_sweep_args(L, w, beta, tau);
   P.a.sched = w.sched;
@@ -784,11 +790,8 @@ nb_status nb_kl_backward(const nb_kl_shape* shape, const void* h_s, const void* 
   }
   if (cudaMemsetAsync(w.sched, 0, size_t(2 * L.n_chunks + 2) * 4, st) != cudaSuccess) return NB_ERR_CUDA;
   launch(compact_kernel, dim3(1), dim3(kScanThreads), 0, st, labels, int(L.N), (long long)shape->ignore_index,
-         w.idx, w.ctrl, (int64_t*)nullptr, grad_out, tau, (int*)nullptr, (long long)L.V, 0ll);
-  launch_gather(L, w, h_s, L.d_s, w.hs, L.lda_s, st, lse_s, lse_t, aux);
-  launch_gather(L, w, h_t, L.d_t, w.ht, L.lda_t, st);
-  launch(zero_masked_rows_kernel, dim3(unsigned(L.N)), dim3(128), 0, st, labels, (long long)shape->ignore_index,
-         dh_s, int(L.d_s));
+         w.idx, w.ctrl, (int64_t*)nullptr, grad_out, tau, (int*)nullptr, (long long)L.V, 0ll, w.inv);
+  launch_gathers(L, w, h_s, h_t, st, lse_s, lse_t, aux);
 
   // one gradient-chunk buffer: per chunk the sweep writes it and the GEMMs then read it, in stream
   // order (two tensor-bound kernels gain nothing from overlapping; serial launches measured faster)
@@ -854,8 +857,9 @@ nb_status nb_kl_backward(const nb_kl_shape* shape, const void* h_s, const void* 
     next_cat(NB_KL_KERNEL_GEMM_BWD);
     launch(gemm_kernel, dim3(pair_grid(dev, tiles)), dim3(kThreads), size_t(kSmemBytes), st, gm, g);
   }
-  launch(scatter_rows_kernel, dim3(unsigned(L.N_pad)), dim3(128), 0, st, (const float*)w.dhc, int(L.d_s), dh_s,
-         (const int*)w.idx, (const Ctrl*)w.ctrl);
+  // every row of dh_s: its compacted row, or zeros for a masked position
+  launch(place_dh_kernel, dim3(unsigned(L.N)), dim3(128), 0, st, (const float*)w.dhc, int(L.d_s), dh_s,
+         (const int*)w.inv);
   return check_launch();
 }
 

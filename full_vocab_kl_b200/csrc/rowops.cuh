@@ -17,9 +17,12 @@ struct Ctrl {          // first bytes of every workspace
 };
 
 // ------------------------------------------------------------------ compaction (one block)
-// Stable list of valid rows: idx[i] = position of the i-th label != ignore_index. With
+// Stable list of valid rows: idx[i] = position of the i-th label != ignore_index. Each of the
+// 32 warps owns one contiguous segment of the labels and reads it in coalesced runs of 32: a
+// count pass (warp ballots), a scan of the 32 segment counts, a placement pass. With
 // `row_label`, also the label of each valid row as a column of the vocabulary range
-// [v_off, v_off + V) held here (-1 outside it).
+// [v_off, v_off + V) held here (-1 outside it); with `inv`, the compacted index of every
+// position (-1 for a masked one).
 constexpr int kScanThreads = 1024;
 
 __global__ void __launch_bounds__(kScanThreads) compact_kernel(const int64_t* __restrict__ labels, int N,
@@ -27,43 +30,46 @@ __global__ void __launch_bounds__(kScanThreads) compact_kernel(const int64_t* __
                                                                Ctrl* ctrl, int64_t* n_valid_out,
                                                                const float* grad_out, float tau,
                                                                int* __restrict__ row_label, long long V,
-                                                               long long v_off) {
+                                                               long long v_off, int* __restrict__ inv) {
   pdl_wait();
   pdl_launch_dependents();
-  __shared__ int warp_sums[32];
+  __shared__ int warp_off[32];
   __shared__ int s_total;
-  const int per = (N + kScanThreads - 1) / kScanThreads;
-  const int b = threadIdx.x * per, e = min(N, b + per);
-  int cnt = 0;
-  for (int i = b; i < e; ++i) cnt += (labels[i] != ignore_index);
-  // block exclusive scan of cnt
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  int incl = cnt;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const int y = __shfl_up_sync(0xffffffffu, incl, o);
-    if (lane >= o) incl += y;
+  const int seg = ((N + 31) / 32 + 31) & ~31;   // labels per warp, a multiple of 32
+  const int b = min(N, warp * seg), e = min(N, b + seg);
+  int cnt = 0;
+  for (int base = b; base < e; base += 32) {
+    const int i = base + lane;
+    cnt += __popc(__ballot_sync(0xffffffffu, i < e && labels[i] != ignore_index));
   }
-  if (lane == 31) warp_sums[warp] = incl;
+  if (lane == 0) warp_off[warp] = cnt;
   __syncthreads();
-  if (warp == 0) {
-    int ws = warp_sums[lane];
-    int wi = ws;
+  if (warp == 0) {   // exclusive scan of the 32 segment counts
+    const int c = warp_off[lane];
+    int incl = c;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
-      const int y = __shfl_up_sync(0xffffffffu, wi, o);
-      if (lane >= o) wi += y;
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
     }
-    warp_sums[lane] = wi - ws;
-    if (lane == 31) s_total = wi;
+    warp_off[lane] = incl - c;
+    if (lane == 31) s_total = incl;
   }
   __syncthreads();
-  int pos = warp_sums[warp] + incl - cnt;
-  for (int i = b; i < e; ++i) {
-    const long long y = labels[i];
-    if (y == ignore_index) continue;
-    if (row_label) row_label[pos] = (y >= v_off && y - v_off < V) ? int(y - v_off) : -1;
-    idx[pos++] = i;
+  int pos = warp_off[warp];
+  for (int base = b; base < e; base += 32) {
+    const int i = base + lane;
+    const long long y = i < e ? labels[i] : ignore_index;
+    const bool v = i < e && y != ignore_index;
+    const unsigned m = __ballot_sync(0xffffffffu, v);
+    const int p = pos + __popc(m & ((1u << lane) - 1u));
+    if (v) {
+      idx[p] = i;
+      if (row_label) row_label[p] = (y >= v_off && y - v_off < V) ? int(y - v_off) : -1;
+    }
+    if (inv && i < e) inv[i] = v ? p : -1;
+    pos += __popc(m);
   }
   if (threadIdx.x == 0) {
     const int nv = s_total;
@@ -74,13 +80,19 @@ __global__ void __launch_bounds__(kScanThreads) compact_kernel(const int64_t* __
 }
 
 // ------------------------------------------------------------------ gather of valid rows
-// dst row i (< n_valid) = src row idx[i] as bf16, zero-padded to `lda` columns; rows
-// n_valid .. round_up(n_valid, 256) (the last pair tile) are zeroed. With `split`, an fp32 source is stored as
-// [hi | lo] with hi = bf16(x) and lo = bf16(x - hi), each half `half` columns wide, so that
-// hi*W + lo*W carries x to about 16 bits.
+// Both models in one launch (blockIdx.y: 0 student, 1 teacher). dst row i (< n_valid) = src row
+// idx[i] as bf16, zero-padded to `lda` columns; rows n_valid .. round_up(n_valid, 256) (the last
+// pair tile) are zeroed. With `split`, an fp32 source is stored as [hi | lo] with hi = bf16(x) and
+// lo = bf16(x - hi), each half `half` columns wide, so that hi*W + lo*W carries x to about 16 bits.
+struct GatherSrc {
+  const void* src;
+  int d, lda, half;
+  __nv_bfloat16* dst;
+};
+
 template <bool F32_SRC>
-__global__ void gather_rows_kernel(const void* __restrict__ src, int d, __nv_bfloat16* __restrict__ dst, int lda,
-                                   int half, const int* __restrict__ idx, const Ctrl* __restrict__ ctrl,
+__global__ void gather_rows_kernel(GatherSrc g0, GatherSrc g1, const int* __restrict__ idx,
+                                   const Ctrl* __restrict__ ctrl,
                                    // optional per-row constants (backward): base-2 LSEs and aux
                                    const float* lse_s, const float* lse_t, const float* aux, float* row_l2s,
                                    float* row_l2t, float* row_aux) {
@@ -90,30 +102,31 @@ __global__ void gather_rows_kernel(const void* __restrict__ src, int d, __nv_bfl
   const int nv = ctrl->n_valid;
   const int rows_needed = ((nv + kPairM - 1) / kPairM) * kPairM;
   if (i >= rows_needed) return;
-  __nv_bfloat16* out = dst + (long long)i * lda;
+  const GatherSrc g = blockIdx.y ? g1 : g0;
+  __nv_bfloat16* out = g.dst + (long long)i * g.lda;
   const bool live = i < nv;
   const int r = live ? idx[i] : 0;
-  if (row_l2s && threadIdx.x == 0) {
+  if (row_l2s && blockIdx.y == 0 && threadIdx.x == 0) {
     row_l2s[i] = live ? lse_s[r] * kLog2e : 0.f;
     row_l2t[i] = live ? lse_t[r] * kLog2e : 0.f;
     row_aux[i] = live ? aux[r] : 0.f;
   }
   if (!F32_SRC) {
-    const __nv_bfloat16* in = static_cast<const __nv_bfloat16*>(src) + (long long)r * d;
+    const __nv_bfloat16* in = static_cast<const __nv_bfloat16*>(g.src) + (long long)r * g.d;
     // d is a multiple of 8: 16-byte vectors
-    for (int c = threadIdx.x * 8; c < lda; c += blockDim.x * 8) {
+    for (int c = threadIdx.x * 8; c < g.lda; c += blockDim.x * 8) {
       uint4 v = make_uint4(0, 0, 0, 0);
-      if (live && c < d) v = *reinterpret_cast<const uint4*>(in + c);
+      if (live && c < g.d) v = *reinterpret_cast<const uint4*>(in + c);
       *reinterpret_cast<uint4*>(out + c) = v;
     }
   } else {
-    const float* in = static_cast<const float*>(src) + (long long)r * d;
-    for (int c = threadIdx.x; c < half; c += blockDim.x) {
-      float x = (live && c < d) ? in[c] : 0.f;
+    const float* in = static_cast<const float*>(g.src) + (long long)r * g.d;
+    for (int c = threadIdx.x; c < g.half; c += blockDim.x) {
+      float x = (live && c < g.d) ? in[c] : 0.f;
       const __nv_bfloat16 hi = __float2bfloat16_rn(x);
       const __nv_bfloat16 lo = __float2bfloat16_rn(x - __bfloat162float(hi));
       out[c] = hi;
-      out[half + c] = lo;
+      out[g.half + c] = lo;
     }
   }
 }
@@ -127,10 +140,10 @@ __global__ void gather_rows_kernel(const void* __restrict__ src, int d, __nv_bfl
 // With `side`, the student's entropy and label log-probability are written as well:
 //   H = ln 2 * (log2 l_s - E / l_s), E = sum_k 2^(m_k - M) (e_k + (m_k - M) l_k)
 //   log S[label] = ln 2 * (x_label - L2_s)  (NaN when the sweep saw no label column)
-// Block = 32 rows x 8 split lanes: lane j of row r visits splits j, j + 8, ... so that a warp
-// (32 consecutive rows, one split) reads contiguous memory; the 8 partial results of a row
+// Block = 32 rows x 16 split lanes: lane j of row r visits splits j, j + 16, ... so that a warp
+// (32 consecutive rows, one split) reads contiguous memory; the 16 partial results of a row
 // are combined in shared memory in a fixed order.
-constexpr int kMergeRows = 32, kMergeLanes = 8;
+constexpr int kMergeRows = 32, kMergeLanes = 16;
 
 __global__ void __launch_bounds__(kMergeRows * kMergeLanes)
     merge_kernel(const float* __restrict__ state, long long fs, int ld, int n_split, const int* __restrict__ idx,
@@ -148,6 +161,7 @@ __global__ void __launch_bounds__(kMergeRows * kMergeLanes)
   const bool live = i < nv;
   float ms = kNegBig, mt = kNegBig;
   if (live)
+#pragma unroll 2
     for (int k = j; k < n_split; k += kMergeLanes) {
       ms = fmaxf(ms, state[(long long)k * ld + i]);
       mt = fmaxf(mt, state[2 * fs + (long long)k * ld + i]);
@@ -163,6 +177,7 @@ __global__ void __launch_bounds__(kMergeRows * kMergeLanes)
   }
   double ls = 0.0, lt = 0.0, a = 0.0, e = 0.0;
   if (live)
+#pragma unroll 2
     for (int k = j; k < n_split; k += kMergeLanes) {
       const long long o = (long long)k * ld + i;
       const double fs_ = exp2f(state[o] - ms);
@@ -407,27 +422,21 @@ __global__ void __launch_bounds__(1024) mean_kernel(const float* __restrict__ lo
   }
 }
 
-// dh_s[idx[i]] = dh_c[i] for the valid rows (the GEMMs accumulate into the compacted dh_c).
-__global__ void scatter_rows_kernel(const float* __restrict__ src, int d, float* __restrict__ dst,
-                                    const int* __restrict__ idx, const Ctrl* __restrict__ ctrl) {
+// dh_s row r = dh_c[inv[r]] for a valid position (the GEMMs accumulate into the compacted dh_c),
+// zeros for a masked one.
+__global__ void place_dh_kernel(const float* __restrict__ dhc, int d, float* __restrict__ dh,
+                                const int* __restrict__ inv) {
   pdl_wait();
   pdl_launch_dependents();
-  const int i = blockIdx.x;
-  if (i >= ctrl->n_valid) return;
-  const float4* in = reinterpret_cast<const float4*>(src + (long long)i * d);
-  float4* out = reinterpret_cast<float4*>(dst + (long long)idx[i] * d);
-  for (int c = threadIdx.x; c < d / 4; c += blockDim.x) out[c] = in[c];
-}
-
-// Zero the dh_s rows of masked positions (valid rows are written by the scatter).
-__global__ void zero_masked_rows_kernel(const int64_t* __restrict__ labels, long long ignore_index, float* dh,
-                                        int d) {
-  pdl_wait();
-  pdl_launch_dependents();
-  const int r = blockIdx.x;
-  if (labels[r] != ignore_index) return;
-  float* row = dh + (long long)r * d;
-  for (int c = threadIdx.x; c < d; c += blockDim.x) row[c] = 0.f;
+  const long long r = blockIdx.x;
+  const int k = inv[r];
+  float4* out = reinterpret_cast<float4*>(dh + r * d);
+  if (k < 0) {
+    for (int c = threadIdx.x; c < d / 4; c += blockDim.x) out[c] = make_float4(0.f, 0.f, 0.f, 0.f);
+  } else {
+    const float4* in = reinterpret_cast<const float4*>(dhc + (long long)k * d);
+    for (int c = threadIdx.x; c < d / 4; c += blockDim.x) out[c] = in[c];
+  }
 }
 
 // ------------------------------------------------------------------ spectral basis selection
