@@ -37,6 +37,11 @@ constexpr int kThreads = 128 + kEpiThreads;            // warpgroup 0: TMA warp,
 constexpr int kRegsLaunch = 168;
 constexpr int kRegsCtl = 56;
 constexpr int kRegsEpi = 224;
+
+// Which roles wait with sleeping barrier tests (descheduled until the phase completes) rather
+// than by polling: the epilogue warps spend most of a tile waiting for an accumulator.
+constexpr bool kSweepSleepEpi = true, kSweepSleepProducer = true, kSweepSleepMma = true;
+constexpr bool kGemmSleepEpi = true, kGemmSleepProducer = true, kGemmSleepMma = true;
 static_assert(128 * kRegsCtl + kEpiThreads * kRegsEpi <= kThreads * kRegsLaunch, "register split");
 constexpr int kHalfN = kBlockN / 2;                    // columns per epilogue thread per tile
 // Per epilogue warp, one 4 KB staging buffer for TMA stores (32 rows x 128 bytes, 128-byte

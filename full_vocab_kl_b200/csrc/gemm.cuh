@@ -104,8 +104,8 @@ __device__ __forceinline__ void gemm_producer(const GemmMaps& maps, const GemmAr
     if (rank == 0) {
       tile = next_work(p.sched, it);
       if (tile >= nt) tile = -1;
-      if (!ring_put(s, it, tile, w)) { ok = false; break; }
-    } else if (!ring_get(s, it, tile, w, false)) {
+      if (!ring_put<kGemmSleepProducer>(s, it, tile, w)) { ok = false; break; }
+    } else if (!ring_get<kGemmSleepProducer>(s, it, tile, w, false)) {
       ok = false;
       break;
     }
@@ -114,7 +114,7 @@ __device__ __forceinline__ void gemm_producer(const GemmMaps& maps, const GemmAr
     const GemmProb& q = p.prob[ti.prob];
     const int am0 = ti.m0 + int(rank) * kBlockM, bn0 = ti.n0 + int(rank) * kHalfB;
     for (int kb = 0; kb < ti.nkb; ++kb) {
-      if (!mbar_wait_cl(&s.empty[stage], phase ^ 1u, w)) { ok = false; break; }
+      if (!mbar_wait_cl<kGemmSleepProducer>(&s.empty[stage], phase ^ 1u, w)) { ok = false; break; }
       const uint32_t bar = smem_addr(&s.full[stage]);
       if (rank == 0) mbar_arrive_expect_tx(&s.full[stage], p.wide ? kWidePairStageBytes : kPairStageBytes);
       const int kc = kb * kBlockK;
@@ -141,20 +141,21 @@ __device__ __forceinline__ void gemm_mma(const GemmArgs& p, int nv, const SweepS
   bool ok = true;
   for (int it = 0; ok; ++it) {
     int tile;
-    if (!ring_get(s, it, tile, w, false)) { ok = false; break; }
+    if (!ring_get<kGemmSleepMma>(s, it, tile, w, false)) { ok = false; break; }
     if (tile < 0) break;
     const TileInfo ti = tile_info(p, nv, tile);
     const GemmProb& q = p.prob[ti.prob];
     const uint32_t idesc = make_idesc(kPairM, kBlockN, q.a_mn, q.b_mn);
     if (p.wide) {
       // both accumulators hold this tile: columns [n0, n0 + 256) in buffer 0, the next 256 in 1
-      if (!mbar_wait_cl(&s.tempty[0], acc_phase ^ 1u, w) || !mbar_wait_cl(&s.tempty[1], acc_phase ^ 1u, w)) {
+      if (!mbar_wait_cl<kGemmSleepMma>(&s.tempty[0], acc_phase ^ 1u, w) ||
+          !mbar_wait_cl<kGemmSleepMma>(&s.tempty[1], acc_phase ^ 1u, w)) {
         ok = false;
         break;
       }
       tc_fence_after();
       for (int kb = 0; kb < ti.nkb; ++kb) {
-        if (!mbar_wait(&s.full[stage], phase, w)) { ok = false; break; }
+        if (!mbar_wait<kGemmSleepMma>(&s.full[stage], phase, w)) { ok = false; break; }
         const uint32_t sa = stage_a(s, 1, stage);
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
@@ -175,12 +176,12 @@ __device__ __forceinline__ void gemm_mma(const GemmArgs& p, int nv, const SweepS
       acc_phase ^= 1u;
       continue;
     }
-    if (!mbar_wait_cl(&s.tempty[acc], acc_phase ^ 1u, w)) { ok = false; break; }
+    if (!mbar_wait_cl<kGemmSleepMma>(&s.tempty[acc], acc_phase ^ 1u, w)) { ok = false; break; }
     tc_fence_after();
     const uint32_t d = tmem_base + acc * kBlockN;
     for (int kb = 0; kb < ti.nkb; ++kb) {
       // TMA bytes are ordered by the barrier's transaction count: no tcgen05 fence here
-      if (!mbar_wait(&s.full[stage], phase, w)) { ok = false; break; }
+      if (!mbar_wait<kGemmSleepMma>(&s.full[stage], phase, w)) { ok = false; break; }
       const uint32_t sa = stage_a(s, 0, stage);
       const uint32_t sb = stage_b(s, 0, stage, 0);
 #pragma unroll
@@ -219,7 +220,7 @@ __device__ __forceinline__ void gemm_epilogue(const GemmMaps& maps, const GemmAr
   uint32_t acc_phase = 0;
   for (int it = 0;; ++it) {
     int tile;
-    if (!ring_get(s, it, tile, w, true)) return;
+    if (!ring_get<kGemmSleepEpi>(s, it, tile, w, true)) return;
     if (tile < 0) break;
     const TileInfo ti = tile_info(p, nv, tile);
     const GemmProb& q = p.prob[ti.prob];
@@ -228,7 +229,7 @@ __device__ __forceinline__ void gemm_epilogue(const GemmMaps& maps, const GemmAr
 #pragma unroll 1
     for (int sub = 0; sub < (p.wide ? 2 : 1); ++sub) {
     const int n0 = ti.n0 + sub * kBlockN;
-    if (!mbar_wait_cl(&s.tfull[acc], acc_phase, w)) return;
+    if (!mbar_wait_cl<kGemmSleepEpi>(&s.tfull[acc], acc_phase, w)) return;
     tc_fence_after();
     const uint32_t base = tmem_base + lane_addr + acc * kBlockN + half * kHalfN;
 #pragma unroll 1

@@ -33,7 +33,8 @@ namespace {
 
 constexpr unsigned long long kWaitLimitNs = 1000000000ull;  // 1 s per pipeline wait
 constexpr int kTilesPerUnitFwd = 8;                          // 2048 vocabulary columns per unit
-constexpr int kTailItems = 160;   // single-tile work items at the end of a forward sweep (~2 waves of pairs)
+constexpr int kTilesPerUnitGrad = 4;                         // gradient sweep: 1024 columns per unit
+constexpr int kTailItems = 160;   // single-tile work items at the end of a sweep (~2 waves of pairs)
 constexpr size_t kCtrlBytes = 256;
 // Compacted h rows of both models per token group of the sweeps' work order. Each of the B200's two
 // L2 halves keeps its own copy of lines its SMs read, so the rows re-read for every vocabulary tile
@@ -85,6 +86,15 @@ struct Layout {
   long long fs_state;    // elements between state fields
 };
 
+// Vocabulary units of a sweep over n_vt tiles: the first (returned) units are runs of
+// tiles_per_unit tiles, the rest single tiles, enough that the last ~kTailItems work items (over
+// all n_tt token tiles) are short and the launch does not end on long items that leave most CTA
+// pairs idle.
+int big_units(int n_vt, int64_t n_tt, int tiles_per_unit) {
+  const int n_single = int(std::min<int64_t>(n_vt, (kTailItems + n_tt - 1) / n_tt));
+  return (n_vt - n_single) / tiles_per_unit;
+}
+
 bool make_layout(const nb_kl_shape* sh, float beta, Layout& L) {
   if (!sh) return false;
   if (sh->n_tokens < 0 || sh->vocab < 1 || sh->d_s < 8 || sh->d_t < 8) return false;
@@ -105,23 +115,21 @@ bool make_layout(const nb_kl_shape* sh, float beta, Layout& L) {
   L.lda_s = int64_t(L.kb_s) * kBlockK * (L.split ? 2 : 1);
   L.lda_t = int64_t(L.kb_t) * kBlockK * (L.split ? 2 : 1);
   L.n_vt = int((L.V + kBlockN - 1) / kBlockN);
-  // forward units: runs of kTilesPerUnitFwd tiles, then enough single tiles that the last
-  // ~kTailItems work items (over all 256-row token tiles) are short
-  {
-    const int64_t n_tt = L.N_pad / kPairM;
-    const int n_single = int(std::min<int64_t>(L.n_vt, (kTailItems + n_tt - 1) / n_tt));
-    L.n_big = (L.n_vt - n_single) / kTilesPerUnitFwd;
-    const int n_vu = L.n_big + (L.n_vt - L.n_big * kTilesPerUnitFwd);
-    L.n_split = 2 * n_vu;  // two column halves per unit
+  // forward units: runs of kTilesPerUnitFwd tiles, then single tiles
+  L.n_big = big_units(L.n_vt, L.N_pad / kPairM, kTilesPerUnitFwd);
+  L.n_split = 2 * (L.n_big + (L.n_vt - L.n_big * kTilesPerUnitFwd));  // two column halves per unit
+  // default chunk: the vocabulary in equal chunks of at most ~24576 gradient tiles of 128 x 256
+  // (the gradient buffer then takes at most ~1.5 GB whatever the token count; fewer, longer
+  // chunks mean fewer launches and launch tails and fewer re-adds of the compacted dh
+  // accumulator), but at least 4 d_s columns; at most 131072 columns
+  if (sh->chunk_v) {
+    L.chunk_v = sh->chunk_v;
+  } else {
+    const int64_t by_tiles = (int64_t(3) << 21) / (L.N_pad / kBlockM);
+    const int64_t max_chunk = std::max<int64_t>(2048, std::min<int64_t>(131072, std::max<int64_t>(by_tiles, 4 * L.d_s)));
+    const int64_t n_chunks = (L.V + max_chunk - 1) / max_chunk;
+    L.chunk_v = round_up((L.V + n_chunks - 1) / n_chunks, kBlockN);
   }
-  // default chunk: about 16384 gradient tiles of 128 x 256 per sweep launch (the gradient
-  // buffer then takes ~1 GB whatever the token count; longer chunks mean fewer launches, shorter
-  // launch tails and fewer re-adds of the compacted dh accumulator), but at least 4 d_s columns;
-  // between 2048 and 65536 columns
-  const int64_t by_tiles = (int64_t(1) << 22) / (L.N_pad / kBlockM);
-  const int64_t auto_chunk =
-      round_up(std::max<int64_t>(2048, std::min<int64_t>(65536, std::max<int64_t>(by_tiles, 4 * L.d_s))), kBlockN);
-  L.chunk_v = sh->chunk_v ? sh->chunk_v : std::min<int64_t>(auto_chunk, round_up(L.V, kBlockN));
   const bool jsd = beta > 0.f && beta < 1.f;
   size_t off = kCtrlBytes;
   L.off_idx = off;   off = align256(off + size_t(L.N_pad) * 4);
@@ -813,8 +821,7 @@ nb_status nb_kl_backward(const nb_kl_shape* shape, const void* h_s, const void* 
 
   SweepArgs a = base_sweep_args(L, w, beta, tau);
   a.ldG = L.chunk_v;
-  a.tiles_per_unit = 1;
-  a.n_big = 0;
+  a.tiles_per_unit = kTilesPerUnitGrad;
   a.G = w.G;
   GemmArgs g;
   std::memset(&g, 0, sizeof(g));
@@ -843,6 +850,7 @@ nb_status nb_kl_backward(const nb_kl_shape* shape, const void* h_s, const void* 
     const int64_t v0 = int64_t(c) * L.chunk_v, v1 = std::min(L.V, v0 + L.chunk_v);
     a.v_begin = int(v0);
     a.v_end = int(v1);
+    a.n_big = big_units(int((v1 - v0 + kBlockN - 1) / kBlockN), L.N_pad / kPairM, kTilesPerUnitGrad);
     a.sched = w.sched + 2 * c;
     if (beta == 0.f) launch_sweep<kGradFkl>(dev, L, maps, a, st);
     else if (beta == 1.f) launch_sweep<kGradRkl>(dev, L, maps, a, st);

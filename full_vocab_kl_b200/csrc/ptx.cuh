@@ -52,15 +52,32 @@ __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
 }
 
+// Upper bound, in ns, on how long a sleeping test keeps its thread suspended when the phase has
+// not completed: the thread is descheduled until the phase completes (or this time passes)
+// instead of re-polling the barrier, which leaves the issue slots and the power to the warps
+// that do the work. Polling tests (kSleep = false) use the hardware's own short limit.
+constexpr uint32_t kSuspendHintNs = 1000000;
+
+template <bool kSleep = false>
 __device__ __forceinline__ bool mbar_test(uint32_t addr, uint32_t parity) {
   uint32_t done;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(done)
-      : "r"(addr), "r"(parity)
-      : "memory");
+  if (kSleep) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(done)
+        : "r"(addr), "r"(parity), "n"(kSuspendHintNs)
+        : "memory");
+  } else {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(done)
+        : "r"(addr), "r"(parity)
+        : "memory");
+  }
   return done != 0;
 }
 
@@ -70,15 +87,17 @@ struct WaitCtl {
 };
 
 // Wait until the phase with the given parity has completed. Returns false when the
-// time limit runs out (recording the timeout) or when another wait already failed.
+// time limit runs out (recording the timeout) or when another wait already failed. A sleeping
+// wait (kSleep) checks the status word and the clock at least every 16 x kSuspendHintNs.
+template <bool kSleep = false>
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const WaitCtl& w) {
   const uint32_t a = smem_addr(bar);
-  if (mbar_test(a, parity)) return true;
+  if (mbar_test<kSleep>(a, parity)) return true;
   const uint64_t t0 = global_timer_ns();
   for (;;) {
 #pragma unroll 1
     for (int i = 0; i < 16; ++i)
-      if (mbar_test(a, parity)) return true;
+      if (mbar_test<kSleep>(a, parity)) return true;
     if (*reinterpret_cast<volatile int*>(w.status) != 0) return false;
     if (global_timer_ns() - t0 > w.limit_ns) {
       atomicCAS(w.status, 0, kStatusTimeout);
@@ -185,26 +204,38 @@ __device__ __forceinline__ void mbar_arrive_remote(uint32_t cl_addr) {
 __device__ __forceinline__ void st_remote_u32(uint32_t cl_addr, uint32_t v) {
   asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(cl_addr), "r"(v) : "memory");
 }
+template <bool kSleep = false>
 __device__ __forceinline__ bool mbar_test_cluster(uint32_t addr, uint32_t parity) {
   uint32_t done;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(done)
-      : "r"(addr), "r"(parity)
-      : "memory");
+  if (kSleep) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(done)
+        : "r"(addr), "r"(parity), "n"(kSuspendHintNs)
+        : "memory");
+  } else {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(done)
+        : "r"(addr), "r"(parity)
+        : "memory");
+  }
   return done != 0;
 }
 // Bounded wait with cluster-scope acquire (for barriers that the peer CTA arrives on).
+template <bool kSleep = false>
 __device__ __forceinline__ bool mbar_wait_cl(uint64_t* bar, uint32_t parity, const WaitCtl& w) {
   const uint32_t a = smem_addr(bar);
-  if (mbar_test_cluster(a, parity)) return true;
+  if (mbar_test_cluster<kSleep>(a, parity)) return true;
   const uint64_t t0 = global_timer_ns();
   for (;;) {
 #pragma unroll 1
     for (int i = 0; i < 16; ++i)
-      if (mbar_test_cluster(a, parity)) return true;
+      if (mbar_test_cluster<kSleep>(a, parity)) return true;
     if (*reinterpret_cast<volatile int*>(w.status) != 0) return false;
     if (global_timer_ns() - t0 > w.limit_ns) {
       atomicCAS(w.status, 0, kStatusTimeout);

@@ -180,9 +180,10 @@ __device__ __forceinline__ int next_work(int* sched, int it) {
   return sched ? atomicAdd(sched, 1) : pair + it * n_pairs;
 }
 
+template <bool kSleep>
 __device__ __forceinline__ bool ring_put(const SweepSmem& s, int it, int id, const WaitCtl& w) {
   const int k = it % kRing;
-  if (!mbar_wait_cl(&s.ring_empty[k], ((it / kRing) & 1) ^ 1, w)) return false;
+  if (!mbar_wait_cl<kSleep>(&s.ring_empty[k], ((it / kRing) & 1) ^ 1, w)) return false;
   s.ring_slot[k] = id;
   st_remote_u32(cluster_addr(smem_addr(&s.ring_slot[k]), 1), uint32_t(id));
   mbar_arrive(&s.ring_full[k]);
@@ -191,9 +192,10 @@ __device__ __forceinline__ bool ring_put(const SweepSmem& s, int it, int id, con
 }
 
 // `warp_wide`: every lane waits and reads, lane 0 arrives once for the warp.
+template <bool kSleep>
 __device__ __forceinline__ bool ring_get(const SweepSmem& s, int it, int& id, const WaitCtl& w, bool warp_wide) {
   const int k = it % kRing;
-  if (!mbar_wait_cl(&s.ring_full[k], (it / kRing) & 1, w)) return false;
+  if (!mbar_wait_cl<kSleep>(&s.ring_full[k], (it / kRing) & 1, w)) return false;
   id = *reinterpret_cast<volatile int*>(&s.ring_slot[k]);
   if (warp_wide) __syncwarp();
   if (!warp_wide || (threadIdx.x % 32) == 0)
@@ -254,8 +256,8 @@ __device__ __forceinline__ void sweep_producer(const SweepMaps& maps, const Swee
     if (rank == 0) {
       u = next_work(p.sched, it);
       if (u >= g.n_units) u = -1;
-      if (!ring_put(s, it, u, w)) { ok = false; break; }
-    } else if (!ring_get(s, it, u, w, false)) {
+      if (!ring_put<kSweepSleepProducer>(s, it, u, w)) { ok = false; break; }
+    } else if (!ring_get<kSweepSleepProducer>(s, it, u, w, false)) {
       ok = false;
       break;
     }
@@ -267,7 +269,7 @@ __device__ __forceinline__ void sweep_producer(const SweepMaps& maps, const Swee
     for (int t = unit_t0(p, vu); t < t_end && ok; ++t) {
       const int v0 = p.v_begin + t * kBlockN + int(rank) * kHalfB;
       for (int kb = 0; kb < nk1 + nk2; ++kb) {
-        if (!mbar_wait_cl(&s.empty[stage], phase ^ 1u, w)) { ok = false; break; }
+        if (!mbar_wait_cl<kSweepSleepProducer>(&s.empty[stage], phase ^ 1u, w)) { ok = false; break; }
         const bool one = kb < nk1;
         const int k = one ? kb : kb - nk1;
         const int kbb = k % (one ? bm1 : bm2);
@@ -296,7 +298,7 @@ __device__ __forceinline__ void sweep_mma(const SweepArgs& p, const UnitGrid& g,
   bool ok = true;
   for (int it = 0; ok; ++it) {
     int u;
-    if (!ring_get(s, it, u, w, false)) { ok = false; break; }
+    if (!ring_get<kSweepSleepMma>(s, it, u, w, false)) { ok = false; break; }
     if (u < 0) break;
     int vu, tt;
     decode_unit(p, g, u, vu, tt);
@@ -307,11 +309,11 @@ __device__ __forceinline__ void sweep_mma(const SweepArgs& p, const UnitGrid& g,
         const int k = one ? kb : kb - nk1;
         if (k == 0) {
           // the accumulator of this model must have been read by both CTAs' epilogues
-          if (!mbar_wait_cl(&s.tempty[one ? 0 : 1], (lt & 1u) ^ 1u, w)) { ok = false; break; }
+          if (!mbar_wait_cl<kSweepSleepMma>(&s.tempty[one ? 0 : 1], (lt & 1u) ^ 1u, w)) { ok = false; break; }
           tc_fence_after();
         }
         // TMA bytes are ordered by the barrier's transaction count: no tcgen05 fence here
-        if (!mbar_wait(&s.full[stage], phase, w)) { ok = false; break; }
+        if (!mbar_wait<kSweepSleepMma>(&s.full[stage], phase, w)) { ok = false; break; }
         const uint32_t d = tmem_base + (one ? 0 : kBlockN);
         const uint32_t sa = stage_a_addr(s, stage);
         const uint32_t sb = stage_b_addr(s, stage);
@@ -542,7 +544,7 @@ __device__ __forceinline__ void sweep_epilogue(const SweepMaps& maps, const Swee
 
   for (int it = 0;; ++it) {
     int u;
-    if (!ring_get(s, it, u, w, true)) return;
+    if (!ring_get<kSweepSleepEpi>(s, it, u, w, true)) return;
     if (u < 0) break;
     int vu, tt;
     decode_unit(p, g, u, vu, tt);
@@ -562,14 +564,14 @@ __device__ __forceinline__ void sweep_epilogue(const SweepMaps& maps, const Swee
     const int t_end = unit_t1(p, vu);
     for (int t = unit_t0(p, vu); t < t_end; ++t, ++lt) {
       const int v0 = p.v_begin + t * kBlockN + half * kHalfN;
-      if (!mbar_wait_cl(&s.tfull[1], lt & 1u, w)) return;   // first model complete
+      if (!mbar_wait_cl<kSweepSleepEpi>(&s.tfull[1], lt & 1u, w)) return;   // first model complete
       tc_fence_after();
       float F[4][32];
 #pragma unroll
       for (int ch = 0; ch < 4; ++ch) tmem_ld32(col1 + ch * 32, F[ch]);
       tmem_wait_ld();
       release_accumulator(&s.tempty[0]);
-      if (!mbar_wait_cl(&s.tfull[0], lt & 1u, w)) return;   // second model complete
+      if (!mbar_wait_cl<kSweepSleepEpi>(&s.tfull[0], lt & 1u, w)) return;   // second model complete
       tc_fence_after();
 #pragma unroll
       for (int ch = 0; ch < 4; ++ch) {

@@ -32,7 +32,7 @@ int main(void) {
   nb_kl_shape big = s;
   big.vocab = 2 * s.vocab;
   CHECK(nb_kl_workspace_size(&big, 1.0f) - ws < (size_t)64 << 20);
-  CHECK(nb_kl_chunk_columns(&s) == 65536);
+  CHECK(nb_kl_chunk_columns(&s) == 76032);
   CHECK(nb_kl_workspace_size(&s, 0.5f) >= ws);
 
   /* an invalid shape gives 0 */

@@ -169,10 +169,12 @@ def test_spectral_argument_errors(L):
 
 def test_chunk_columns(L):
     lib = L.lib()
-    # default: ~16384 gradient tiles of 128 x 256 per launch, at least 4 d_s, in [2048, 65536]
-    assert lib.nb_kl_chunk_columns(L.shape_ptr(shape(L))) == 65536
-    assert lib.nb_kl_chunk_columns(L.shape_ptr(shape(L, N=32768, ds=4096, dt=512))) == 16384
-    assert lib.nb_kl_chunk_columns(L.shape_ptr(shape(L, N=65536, ds=256, dt=256))) == 8192
+    # default: the vocabulary in equal chunks (multiples of 256) of at most ~24576 gradient tiles
+    # of 128 x 256 (but at least 4 d_s and 2048, at most 131072 columns)
+    assert lib.nb_kl_chunk_columns(L.shape_ptr(shape(L))) == 76032                  # 2 x 75968 -> 256
+    assert lib.nb_kl_chunk_columns(L.shape_ptr(shape(L, N=32768, ds=4096, dt=512))) == 21760   # 7 chunks
+    assert lib.nb_kl_chunk_columns(L.shape_ptr(shape(L, N=65536, ds=256, dt=256))) == 11776    # 13 chunks
+    assert lib.nb_kl_chunk_columns(L.shape_ptr(shape(L, N=8192, V=248320, ds=5120, dt=5120))) == 82944
     assert lib.nb_kl_chunk_columns(L.shape_ptr(shape(L, N=256, V=1000, ds=256, dt=256))) == 1024
     # an explicit chunk is kept; an invalid shape gives 0
     assert lib.nb_kl_chunk_columns(L.shape_ptr(shape(L, chunk=4096))) == 4096
