@@ -63,8 +63,20 @@ def test_multi_chunk_backward(beta):
 
 
 def test_many_token_tiles_and_splits():
-    # 1100 rows (9 token tiles), V 5000 (40 vocabulary tiles -> 3 splits)
+    # 1100 rows (800 valid: 4 pair tiles, the last ragged), V 5000 (20 vocabulary tiles, the last
+    # one ragged; every tile its own split)
     x = make_custom(1100, 256, 320, 5000, 1.0, 1.0, n_masked=300, teacher="correlated")
+    full_check(x)
+
+
+@pytest.mark.parametrize("beta", [1.0, 0.0, 0.5])
+def test_multi_tile_units_and_single_tail(beta):
+    """8192 positions (32 token tiles on the host side, so the last ~160 work items are the
+    last 5 vocabulary tiles of each token tile), 5192 valid rows (21 pair tiles, the last
+    ragged), V 4000 (16 vocabulary tiles, the last ragged): the forward and JSD sweeps run one
+    8-tile unit and then single tiles, the gradient sweep two 4-tile units and then single
+    tiles; every row against the oracle."""
+    x = make_custom(8192, 64, 96, 4000, beta, 1.0, n_masked=3000, teacher="correlated")
     full_check(x)
 
 
