@@ -39,7 +39,8 @@ constexpr int kRegsCtl = 56;
 constexpr int kRegsEpi = 224;
 
 // Which roles wait with sleeping barrier tests (descheduled until the phase completes) rather
-// than by polling: the epilogue warps spend most of a tile waiting for an accumulator.
+// than by polling. The MMA issuer's wait for a stage's operands is on the critical path, and a
+// polling wait could see the landed operands up to a microsecond late; every role sleeps.
 constexpr bool kSweepSleepEpi = true, kSweepSleepProducer = true, kSweepSleepMma = true;
 constexpr bool kGemmSleepEpi = true, kGemmSleepProducer = true, kGemmSleepMma = true;
 static_assert(128 * kRegsCtl + kEpiThreads * kRegsEpi <= kThreads * kRegsLaunch, "register split");

@@ -53,9 +53,10 @@ __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
 }
 
 // Upper bound, in ns, on how long a sleeping test keeps its thread suspended when the phase has
-// not completed: the thread is descheduled until the phase completes (or this time passes)
-// instead of re-polling the barrier, which leaves the issue slots and the power to the warps
-// that do the work. Polling tests (kSleep = false) use the hardware's own short limit.
+// not completed: the thread is descheduled until the phase completes (or this time passes).
+// Polling tests (kSleep = false) return after the hardware's own short limit, so a polling wait
+// soon falls through to its status-word read in global memory, and a phase that completes
+// during that read is seen only after it.
 constexpr uint32_t kSuspendHintNs = 1000000;
 
 template <bool kSleep = false>

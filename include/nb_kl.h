@@ -80,8 +80,9 @@ typedef struct nb_kl_shape {
 NB_KL_API size_t nb_kl_workspace_size(const nb_kl_shape* shape, float beta);
 
 /* Vocabulary columns per backward chunk for this shape: shape->chunk_v, or the library's
- * default when it is 0 (about 8192 gradient tiles of 128 x 256 per launch, at least 4 d_s,
- * between 2048 and 32768, at most the vocabulary rounded up to 256). 0 for an invalid shape. */
+ * default when it is 0: the vocabulary cut into equal chunks, each a multiple of 256 columns
+ * of at most max(2048, min(131072, max(24576 gradient tiles of 128 x 256 for the padded token
+ * count, 4 d_s))) columns (at most ~1.5 GB of bf16 gradient chunk). 0 for an invalid shape. */
 NB_KL_API int64_t nb_kl_chunk_columns(const nb_kl_shape* shape);
 
 /* Forward ("Nitrobrew 的两个动作": block GEMMs + online log-sum-exp + KL numerator).
