@@ -60,7 +60,7 @@ SIGNATURES = {
     "nb_kl_device_status": (c_int, [c_void_p, c_void_p]),
     "nb_kl_debug_gemm": (c_int, [c_void_p, c_int, c_void_p, c_int, c_int64, c_int64, c_int64, c_void_p, c_void_p,
                                  c_void_p]),
-    "nb_kl_debug_wait_timeout": (c_int, [c_void_p, c_uint64, c_void_p]),
+    "nb_kl_debug_wait_timeout": (c_int, [c_void_p, c_uint64, c_int, c_void_p]),
     "nb_kl_last_launch_count": (c_int, []),
     "nb_kl_timing_enable": (None, [c_int]),
     "nb_kl_timing_read": (c_int, [c_void_p, c_void_p, c_int]),

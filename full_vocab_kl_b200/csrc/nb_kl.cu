@@ -1065,7 +1065,7 @@ nb_status nb_kl_debug_gemm(const void* A, int a_mn_major, const void* B, int b_m
   return check_launch();
 }
 
-nb_status nb_kl_debug_wait_timeout(void* workspace, uint64_t limit_ns, void* stream) {
+nb_status nb_kl_debug_wait_timeout(void* workspace, uint64_t limit_ns, int sleeping, void* stream) {
   g_launches = 0;
   g_launch_failed = false;
   if (!workspace || !aligned16(workspace)) return NB_ERR_INVALID_ARG;
@@ -1076,7 +1076,7 @@ nb_status nb_kl_debug_wait_timeout(void* workspace, uint64_t limit_ns, void* str
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (cudaMemsetAsync(workspace, 0, kCtrlBytes, st) != cudaSuccess) return NB_ERR_CUDA;
   launch(wait_timeout_kernel, dim3(1), dim3(32), 0, st, &static_cast<Ctrl*>(workspace)->status,
-         (unsigned long long)limit_ns);
+         (unsigned long long)limit_ns, sleeping ? 1 : 0);
   return check_launch();
 }
 

@@ -481,8 +481,9 @@ __global__ void __launch_bounds__(256)
   }
 }
 
-// Test hook: wait on an mbarrier that nothing arrives at, with the given limit.
-__global__ void wait_timeout_kernel(int* status, unsigned long long limit_ns) {
+// Test hook: wait on an mbarrier that nothing arrives at, with the given limit, by polling or
+// with the sleeping tests the pipeline kernels use.
+__global__ void wait_timeout_kernel(int* status, unsigned long long limit_ns, int sleeping) {
   pdl_wait();
   pdl_launch_dependents();
   __shared__ uint64_t bar;
@@ -493,7 +494,8 @@ __global__ void wait_timeout_kernel(int* status, unsigned long long limit_ns) {
   __syncthreads();
   if (threadIdx.x == 0) {
     const WaitCtl w{status, limit_ns};
-    mbar_wait(&bar, 0, w);
+    if (sleeping) mbar_wait<true>(&bar, 0, w);
+    else mbar_wait<false>(&bar, 0, w);
   }
 }
 

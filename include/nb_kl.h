@@ -275,10 +275,12 @@ NB_KL_API nb_status nb_kl_device_status(void* workspace, void* stream);
 NB_KL_API nb_status nb_kl_debug_gemm(const void* A, int a_mn_major, const void* B, int b_mn_major, int64_t M, int64_t N,
                            int64_t K, float* C, void* workspace, void* stream);
 
-/* Launches a kernel whose mbarrier wait can never complete, bounded by limit_ns, so that
- * the timeout path can be exercised without hanging the GPU. Afterwards
- * nb_kl_device_status(workspace) reports NB_ERR_TIMEOUT. workspace: 256 bytes. */
-NB_KL_API nb_status nb_kl_debug_wait_timeout(void* workspace, uint64_t limit_ns, void* stream);
+/* Launches a kernel whose mbarrier wait can never complete, bounded by limit_ns (at most 5 s),
+ * so that the timeout path can be exercised without hanging the GPU: sleeping != 0 waits with
+ * the sleeping barrier tests of the pipeline kernels (the limit is checked every 16 suspensions
+ * of at most 1 ms), sleeping == 0 by polling. Afterwards nb_kl_device_status(workspace) reports
+ * NB_ERR_TIMEOUT. workspace: 256 bytes, device memory. */
+NB_KL_API nb_status nb_kl_debug_wait_timeout(void* workspace, uint64_t limit_ns, int sleeping, void* stream);
 
 /* Number of kernel launches the last forward / backward call on this thread made. */
 NB_KL_API int nb_kl_last_launch_count(void);

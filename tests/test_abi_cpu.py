@@ -121,7 +121,8 @@ def test_debug_entry_argument_errors(L):
                                 ctypes.c_void_p(FAKE[3]), None) == L.NB_ERR_INVALID_ARG
     assert lib.nb_kl_debug_gemm(ctypes.c_void_p(FAKE[0]), 0, ctypes.c_void_p(FAKE[1]), 0, 130, 128, 64,
                                 ctypes.c_void_p(FAKE[2]), ctypes.c_void_p(FAKE[3]), None) == L.NB_ERR_INVALID_ARG
-    assert lib.nb_kl_debug_wait_timeout(None, 1000, None) == L.NB_ERR_INVALID_ARG
+    assert lib.nb_kl_debug_wait_timeout(None, 1000, 0, None) == L.NB_ERR_INVALID_ARG
+    assert lib.nb_kl_debug_wait_timeout(None, 1000, 1, None) == L.NB_ERR_INVALID_ARG
 
 
 def test_python_api_refuses_cpu_tensors(L):
