@@ -183,3 +183,27 @@ def test_empty_input():
     assert float(f["loss_mean"]) == 0.0 and int(f["n_valid"]) == 0
     assert dh.shape == (0, 128) and float(dW.abs().max()) == 0.0
     assert nb.device_status(f["workspace"]) == 0
+
+
+@pytest.mark.parametrize("beta,tau", [(1.0, 1.0), (0.0, 1.0), (0.5, 2.0)])
+def test_one_entry_vocabulary(beta, tau):
+    """V = 1: both distributions are a point mass, so every divergence is 0 and so is its gradient
+    (the 255 other columns of the only vocabulary tile are masked), while each LSE is the single
+    tempered logit, compared with the oracle."""
+    x = make_custom(300, 64, 96, 1, beta, tau, n_masked=44, teacher="independent")
+    got = gu.run_library(x)
+    ref = gu.oracle_all(x)
+    valid = x.labels != -100
+    assert got["n_valid"] == int(valid.sum())
+    assert np.abs(got["loss_tok"][valid]).max() <= 1e-5 and abs(got["loss_mean"]) <= 1e-5
+    for k in ("lse_s", "lse_t"):
+        np.testing.assert_allclose(got[k][valid], ref[k][valid], rtol=gu.TOL_LSE, atol=1e-6)
+    assert np.abs(got["dh_s"]).max() <= 1e-6 and np.abs(got["dW_s"]).max() <= 1e-6
+
+
+@pytest.mark.parametrize("beta", [1.0, 0.0, 0.5])
+def test_single_token(beta):
+    """One position, valid: one 256-row token tile holding a single row, every row against the
+    oracle, forward and backward."""
+    x = make_custom(1, 64, 128, 300, beta, 1.0, n_masked=0, teacher="independent")
+    full_check(x)
