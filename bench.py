@@ -718,10 +718,13 @@ def run_library(args):
             "clocks": clk,
             "scratch_bytes": ws_bytes, "peak_extra_alloc_bytes": int(peak_extra), "chunk_v": chunk_cols,
         }
+    plain = not (args.vocab_parallel or args.front_end or args.handoff or args.side)
+    if rank == 0 and world == 1 and plain and args.sustained > 0:
+        result["sustained"] = measure_sustained(lambda: step(h_s, h_t, labels), ms / args.steps,
+                                                step_flops, args.sustained, dev, local)
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
-    plain = not (args.vocab_parallel or args.front_end or args.handoff or args.side)
     if rank == 0 and world == 1 and plain and args.workload == DEFAULT_WORKLOAD and not args.no_workloads:
         # the other workloads of the method's configuration list, each timed on its own
         del ws, dW, dh, W_s, W_t
@@ -736,6 +739,40 @@ def run_library(args):
     return 0
 
 
+def measure_sustained(step, ms_step, step_flops, seconds, dev, gpu_index):
+    """Throughput under the board's power cap: back-to-back steps for about `seconds`, then a
+    cuBLAS bf16 GEMM (8192 x 8192 x 8192, torch.matmul) loop for as long, each device-timed with
+    its own clock record. The GEMM is a reference point for the same power budget, measured in
+    the same process; it is not part of the loss path."""
+    import torch
+
+    def loop(fn, iters):
+        clocks = ClockSampler(gpu_index)
+        clocks.start()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(iters):
+            fn()
+        e1.record()
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / iters, clocks.stop()
+    iters = max(3, int(seconds * 1e3 / ms_step))
+    ms, clk = loop(step, iters)
+    n = 8192
+    A = torch.randn(n, n, device=dev).to(torch.bfloat16)
+    B = torch.randn(n, n, device=dev).to(torch.bfloat16)
+    torch.matmul(A, B)
+    torch.cuda.synchronize()
+    t0 = time.time()
+    torch.matmul(A, B)
+    torch.cuda.synchronize()
+    g_ms, g_clk = loop(lambda: torch.matmul(A, B), max(3, int(seconds / max(time.time() - t0, 1e-4))))
+    tf, g_tf = step_flops / (ms * 1e-3) / 1e12, 2.0 * n ** 3 / (g_ms * 1e-3) / 1e12
+    return {"seconds": seconds, "steps": iters, "ms_per_step": ms, "tflops": tf, "clocks": clk,
+            "cublas_bf16_gemm": {"shape": [n, n, n], "tflops": g_tf, "clocks": g_clk},
+            "tflops_vs_cublas": tf / g_tf}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -746,6 +783,9 @@ def main():
     ap.add_argument("--impl", default="library", choices=["library", "reference"])
     ap.add_argument("--chunk-v", type=int, default=0, help="backward vocabulary chunk (0: library default)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--sustained", type=float, default=0.0,
+                    help="also run about this many seconds of back-to-back steps, then as long a cuBLAS "
+                         "bf16 GEMM loop, under the power cap (0: off)")
     ap.add_argument("--no-workloads", action="store_true",
                     help="skip the device-timed lines of the other workloads (long_jsd, large_vocab, spectral)")
     ap.add_argument("--workload-steps", type=int, default=10, help="timed steps of each other workload")
